@@ -1,0 +1,134 @@
+/*
+ * tl.h -- C ABI of libternary: the ternary linear layer y = alpha * (T x) on
+ * one NVIDIA B200 (sm_100a), with T in {-1, 0, 1} packed losslessly at
+ * 2 bits (4 trits per byte) or 1.6 bits (5 trits per byte).
+ *
+ * Defining passages ("Pith review of Spectra 1.1: Scaling Laws and
+ * Efficient Inference for Ternary Language Models", pith.science):
+ *   - "What carries the argument": a ternary linear layer is a linear layer
+ *     whose weight matrix is restricted to {-1,0,1} times one shared
+ *     floating-point scale; k trits fit p bits when 2^p > 3^k, so 5 trits
+ *     fit one byte (1.6 bits per weight).
+ *   - "Core claim": lossless packing at 2 bits by a base-4 encoding and at
+ *     1.6 bits by a base-3 encoding.
+ *   - Referee report, minor comment 5 (paper section 3.2): decoding by
+ *     running quotients; the partial final block is left open.
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - Trit t is stored as digit d = t + 1 (so -1 -> 0, 0 -> 1, +1 -> 2).
+ *   - T is N x K (output rows x reduction).  Row n of T is packed into row n
+ *     of P, row stride ldp bytes.  Trit k of a row is digit (k mod g) of byte
+ *     floor(k / g), g = 4 (2-bit) or 5 (1.6-bit); digit i has weight b^i,
+ *     b = 4 or 3 (least-significant digit first).
+ *     2-bit:   byte = d0 + 4 d1 + 16 d2 + 64 d3  (a field value 3 is invalid)
+ *     1.6-bit: byte = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4  (bytes >= 243 invalid)
+ *   - A partial last byte is completed with 0-trits (digit 1).  Bytes in
+ *     [row_bytes, ldp) are written as 0 by the packers and never interpreted.
+ *   - X is M x K, Y is M x N, both IEEE binary16 (passed as uint16_t bit
+ *     patterns), row-major with row strides ldx / ldy elements:
+ *     Y[m][n] = fp16_rn(alpha * sum_k T[n][k] * X[m][k]), the sum taken in
+ *     fp32 (products are exact; the order of the additions is unspecified).
+ *
+ * All functions return a status code (TL_OK = 0) and never throw.  They
+ * keep no state between calls except a per-device error word set by the
+ * kernels' bounded waits (see tl_device_status) and lazily created
+ * per-device launch parameters; they are safe to call concurrently from
+ * several host threads on different streams.
+ */
+#ifndef TERNARY_TL_H
+#define TERNARY_TL_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TL_FMT_2BIT 2    /* 4 trits per byte, base 4 */
+#define TL_FMT_1P6BIT 16 /* 5 trits per byte, base 3 */
+
+#define TL_GEMV_MAX_M 8   /* tl_gemv: 1 <= M <= 8 */
+#define TL_GEMM_MIN_M 16  /* tl_gemm: M >= 16 */
+
+enum tl_status {
+    TL_OK = 0,
+    TL_ERR_INVALID_ARG = 1, /* null pointer, size out of range, bad format, bad stride */
+    TL_ERR_BAD_TRIT = 2,    /* a trit outside {-1, 0, 1} given to a packer */
+    TL_ERR_BAD_CODE = 3,    /* a byte that is not a valid code given to tl_unpack */
+    TL_ERR_ALIGN = 4,       /* a device pointer or stride breaks the alignment rules */
+    TL_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
+    TL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (see tl_device_status) */
+    TL_ERR_UNSUPPORTED = 7  /* no kernel for this (format, shape) on this device */
+};
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *tl_status_str(int status);
+
+/* The CUDA error code (cudaError_t value) behind the last TL_ERR_CUDA
+ * returned on the calling host thread, or 0. */
+int tl_last_cuda_error(void);
+
+/* Bytes per packed row: ceil(K / 4) for TL_FMT_2BIT, ceil(K / 5) for
+ * TL_FMT_1P6BIT.  Returns -1 for an unknown format or K < 0.  Pure. */
+int64_t tl_packed_row_bytes(int fmt, int64_t K);
+
+/* Pack int8 trits T[N][ldt] (host memory) into P[N][ldp] (host memory) at
+ * 2 bits per trit ("Core claim": base-4 encoding).  Requires ldt >= K and
+ * ldp >= tl_packed_row_bytes(TL_FMT_2BIT, K); P must hold N * ldp bytes and
+ * may not overlap T.  Every trit must be -1, 0 or 1, else TL_ERR_BAD_TRIT
+ * and P is left unspecified.  The caller owns both buffers; nothing is
+ * allocated.  N == 0 or K == 0 is valid (pads only). */
+int tl_pack2(const int8_t *T, int64_t N, int64_t K, int64_t ldt, uint8_t *P, int64_t ldp);
+
+/* The same at 1.6 bits per trit ("What carries the argument": 5 trits in
+ * one byte, base 3, valid since 3^5 = 243 <= 2^8).  ldp >=
+ * tl_packed_row_bytes(TL_FMT_1P6BIT, K). */
+int tl_pack16(const int8_t *T, int64_t N, int64_t K, int64_t ldt, uint8_t *P, int64_t ldp);
+
+/* Unpack P[N][ldp] (host) into int8 trits T[N][ldt] (host), the map U of
+ * the packing theorem (U(P(t)) = t, "Circularity Check").  Every byte in
+ * [0, row_bytes) of every row is validated: a 2-bit byte with a field equal
+ * to 3, or a 1.6-bit byte >= 243, returns TL_ERR_BAD_CODE and, when
+ * bad_index is not NULL, stores the offset n * ldp + j of the first such
+ * byte in row-major order (T is then partly written).  Digits of the last
+ * byte beyond K and bytes past row_bytes are not returned. */
+int tl_unpack(int fmt, const uint8_t *P, int64_t N, int64_t K, int64_t ldp, int8_t *T,
+              int64_t ldt, int64_t *bad_index);
+
+/* Decode-shaped layer, 1 <= M <= TL_GEMV_MAX_M:
+ *   Y[m][n] = fp16_rn(alpha * sum_k T[n][k] X[m][k]),  m < M, n < N.
+ * dT: packed T on the device, N rows of ldp bytes, format fmt.
+ * dX: binary16 activations on the device, M rows of ldx elements.
+ * dY: binary16 outputs on the device, M rows of ldy elements; every
+ *     element m < M, n < N is overwritten (no accumulation into Y).
+ * alpha: the layer's shared scale ("What carries the argument").
+ * stream: a cudaStream_t (NULL = the legacy default stream).
+ * Rules: dT, dX, dY 16-byte aligned; ldp % 16 == 0 and ldp >= row bytes;
+ * ldx % 8 == 0, ldx >= K; ldy % 8 == 0, ldy >= N; N >= 1, K >= 1 (else
+ * TL_ERR_INVALID_ARG / TL_ERR_ALIGN before anything is enqueued).  The
+ * kernels read only [0, ldp) of each packed row, X[m][0..ldx) and write
+ * only Y[m][0..N).  The call is asynchronous and stream-ordered: it returns
+ * once the work is enqueued, allocates nothing and does not synchronize.
+ * Codes are not validated on the device: an invalid byte yields an
+ * unspecified (but finite-time, in-bounds) result.  The buffers are the
+ * caller's and must stay valid until the stream reaches this work. */
+int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+            int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream);
+
+/* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and
+ * rules as tl_gemv (tensor-core kernel: packed tiles are expanded to fp16
+ * on chip and multiplied with tcgen05 MMAs accumulating in fp32). */
+int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+            int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream);
+
+/* Synchronizes `stream`, then reads and clears the current device's error
+ * word, which kernels set when one of their bounded waits gives up instead
+ * of spinning forever.  Returns TL_OK, TL_ERR_TIMEOUT, or TL_ERR_CUDA if
+ * the synchronization itself failed. */
+int tl_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TERNARY_TL_H */

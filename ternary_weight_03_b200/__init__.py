@@ -1,0 +1,173 @@
+"""Python binding of libternary (ctypes; argument marshalling only).
+
+Every step of the layer runs inside ``libternary.so``: the host codec
+(tl_pack2 / tl_pack16 / tl_unpack) and the sm_100a kernels (tl_gemv,
+tl_gemm).  PyTorch is used only for device buffers and streams.  There is no
+fallback: if the library is missing or a call fails, an exception is raised.
+
+Functions take numpy arrays (host codec) or torch CUDA tensors (layer calls).
+Activations and outputs are fp16; packed weights are uint8 [N, ldp].
+"""
+from __future__ import annotations
+
+import ctypes
+from pathlib import Path
+
+import numpy as np
+
+PKG = Path(__file__).resolve().parent
+LIB_PATH = PKG / "libternary.so"
+
+FMT_2BIT = 2
+FMT_1P6BIT = 16
+GEMV_MAX_M = 8
+GEMM_MIN_M = 16
+
+STATUS = {0: "TL_OK", 1: "TL_ERR_INVALID_ARG", 2: "TL_ERR_BAD_TRIT", 3: "TL_ERR_BAD_CODE",
+          4: "TL_ERR_ALIGN", 5: "TL_ERR_CUDA", 6: "TL_ERR_TIMEOUT", 7: "TL_ERR_UNSUPPORTED"}
+
+# (name, restype, argtypes) of every symbol the C header declares
+_i64, _i32, _p, _f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
+SIGNATURES = {
+    "tl_status_str": (ctypes.c_char_p, [_i32]),
+    "tl_last_cuda_error": (_i32, []),
+    "tl_packed_row_bytes": (_i64, [_i32, _i64]),
+    "tl_pack2": (_i32, [_p, _i64, _i64, _i64, _p, _i64]),
+    "tl_pack16": (_i32, [_p, _i64, _i64, _i64, _p, _i64]),
+    "tl_unpack": (_i32, [_i32, _p, _i64, _i64, _i64, _p, _i64, ctypes.POINTER(_i64)]),
+    "tl_gemv": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _p]),
+    "tl_gemm": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _p]),
+    "tl_device_status": (_i32, [_p]),
+}
+
+
+class TLError(RuntimeError):
+    def __init__(self, fn: str, status: int, cuda: int = 0):
+        self.status = status
+        msg = f"{fn} returned {STATUS.get(status, status)}"
+        if cuda:
+            msg += f" (cudaError {cuda})"
+        super().__init__(msg)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libternary.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not LIB_PATH.exists():
+            raise RuntimeError(f"libternary.so not found at {LIB_PATH}: run "
+                               "`python -m ternary_weight_03_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(str(LIB_PATH))
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != 0:
+        raise TLError(fn, rc, lib().tl_last_cuda_error() if rc == 5 else 0)
+
+
+def status_str(rc: int) -> str:
+    return lib().tl_status_str(rc).decode()
+
+
+def row_bytes(fmt: int, K: int) -> int:
+    return int(lib().tl_packed_row_bytes(fmt, K))
+
+
+def padded_ldp(fmt: int, K: int, align: int = 16) -> int:
+    """The smallest legal device row stride: row bytes rounded up to 16."""
+    rb = row_bytes(fmt, K)
+    return max(align, (rb + align - 1) // align * align)
+
+
+# -- host codec -----------------------------------------------------------------
+def pack(fmt: int, T: np.ndarray, ldp: int | None = None, out: np.ndarray | None = None) -> np.ndarray:
+    """Pack int8 trits [N, K] into uint8 [N, ldp] (ldp defaults to padded_ldp)."""
+    T = np.ascontiguousarray(T, dtype=np.int8)
+    N, K = T.shape
+    ldp = padded_ldp(fmt, K) if ldp is None else ldp
+    if out is None:
+        out = np.empty((N, ldp), dtype=np.uint8)
+    assert out.dtype == np.uint8 and out.flags.c_contiguous and out.shape == (N, ldp)
+    fn = lib().tl_pack2 if fmt == FMT_2BIT else lib().tl_pack16
+    if fmt not in (FMT_2BIT, FMT_1P6BIT):
+        raise TLError("pack", 1)
+    _check("tl_pack", fn(T.ctypes.data, N, K, K, out.ctypes.data, ldp))
+    return out
+
+
+def unpack(fmt: int, P: np.ndarray, K: int) -> np.ndarray:
+    """Unpack uint8 [N, ldp] into int8 trits [N, K]; raises TLError on a bad code."""
+    P = np.ascontiguousarray(P, dtype=np.uint8)
+    N, ldp = P.shape
+    T = np.empty((N, max(K, 1)), dtype=np.int8)
+    bad = _i64(-1)
+    rc = lib().tl_unpack(fmt, P.ctypes.data, N, K, ldp, T.ctypes.data, max(K, 1), ctypes.byref(bad))
+    if rc != 0:
+        err = TLError("tl_unpack", rc)
+        err.bad_index = int(bad.value)
+        raise err
+    return T[:, :K]
+
+
+# -- device layer ---------------------------------------------------------------
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _layer(fn_name: str, fmt: int, dT, alpha: float, X, K: int, out=None, stream=None, M=None):
+    import torch
+    assert dT.is_cuda and dT.dtype == torch.uint8 and dT.dim() == 2
+    assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2
+    N, ldp = dT.shape
+    M = X.shape[0] if M is None else M
+    if out is None:
+        out = torch.empty((M, N + (-N) % 8), dtype=torch.float16, device=X.device)
+    assert out.is_cuda and out.dtype == torch.float16
+    rc = getattr(lib(), fn_name)(fmt, dT.data_ptr(), dT.stride(0), float(alpha), X.data_ptr(),
+                                 X.stride(0), out.data_ptr(), out.stride(0), M, N, K,
+                                 _stream_ptr(stream))
+    _check(fn_name, rc)
+    return out[:, :N]
+
+
+def gemv(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None):
+    """Y[M, N] = alpha * X T^T for 1 <= M <= 8 (decode-shaped)."""
+    return _layer("tl_gemv", fmt, dT, alpha, X, K, out, stream)
+
+
+def gemm(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None):
+    """Y[M, N] = alpha * X T^T for M >= 16 (tensor-core GEMM)."""
+    return _layer("tl_gemm", fmt, dT, alpha, X, K, out, stream)
+
+
+def linear(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None):
+    """Dispatch on M: tl_gemv for M <= 8, two tl_gemv calls (8 + rest) for
+    9 <= M <= 15, tl_gemm for M >= 16."""
+    import torch
+    M = X.shape[0]
+    if M <= GEMV_MAX_M:
+        return gemv(fmt, dT, alpha, X, K, out, stream)
+    if M < GEMM_MIN_M:
+        N = dT.shape[0]
+        if out is None:
+            out = torch.empty((M, N + (-N) % 8), dtype=torch.float16, device=X.device)
+        gemv(fmt, dT, alpha, X[:GEMV_MAX_M], K, out[:GEMV_MAX_M], stream)
+        gemv(fmt, dT, alpha, X[GEMV_MAX_M:], K, out[GEMV_MAX_M:], stream)
+        return out[:, :N]
+    return gemm(fmt, dT, alpha, X, K, out, stream)
+
+
+def device_status(stream=None) -> int:
+    return int(lib().tl_device_status(_stream_ptr(stream)))
