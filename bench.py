@@ -1,0 +1,619 @@
+#!/usr/bin/env python3
+"""Benchmark of the ternary linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Headline workload (one "step"): the decode GEMV sweep with 2-bit packing:
+(K, N) in {(3072,3072), (3072,8192), (8192,3072), (4096,4096), (4096,14336),
+(14336,4096)}, M in {1, 8}: twelve tl_gemv calls, fp16 activations ~ N(0,1),
+uniform trits, one alpha ~ U(0.01, 0.05) per matrix, seeds 0..5.  Every call
+reads a different copy of its packed matrix; the copies rotate through more
+than three times the L2 size, so every weight byte comes from HBM.  A step is
+one CUDA-graph replay of the twelve calls (event records between them give
+the per-launch kernel times).
+
+Metric: packed-weight bytes streamed per second (GB/s), whole job, i.e. the
+sum over ranks of bytes divided by the slowest rank's time.  Under torchrun
+every rank runs the same sweep on its own GPU (weak scaling; the layer needs
+no collective).  Secondary measurements (1.6-bit sweep, batched GEMM,
+30-layer decode step) are appended under "secondary".
+
+--impl reference times the CPU oracle (the definition of the layer, in
+double) on a bounded sample of the same workload; it is the baseline arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+from pathlib import Path
+
+import numpy as np
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+SWEEP = [(3072, 3072), (3072, 8192), (8192, 3072), (4096, 4096), (4096, 14336), (14336, 4096)]
+SWEEP_M = (1, 8)
+L2_BYTES = 126 << 20
+METRIC = "packed-ternary GEMV HBM GB/s (% of peak); batched GEMM TFLOP/s (% peak)"
+WORKLOAD = ("decode GEMV sweep, 2-bit packing, M in {1,8}, (K,N) in (3072,3072) (3072,8192) "
+            "(8192,3072) (4096,4096) (4096,14336) (14336,4096), fp16 x ~ N(0,1), uniform trits, "
+            "alpha ~ U(0.01,0.05) per matrix, seeds 0..5")
+DECODE_LAYER = [("q", 3072, 3072), ("k", 3072, 3072), ("v", 3072, 3072), ("o", 3072, 3072),
+                ("gate", 3072, 8192), ("up", 3072, 8192), ("down", 8192, 3072)]
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (testable with gloo on CPU)
+# ---------------------------------------------------------------------------
+def dist_env():
+    """(rank, local_rank, world) from the torchrun environment, else (0, 0, 1)."""
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def reduce_step_time(ms: float, units: float, group=None):
+    """Max of the per-rank elapsed time and sum of per-rank work units."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return ms, units
+    t = torch.tensor([ms], dtype=torch.float64)
+    u = torch.tensor([units], dtype=torch.float64)
+    if dist.get_backend(group) == "nccl":
+        t, u = t.cuda(), u.cuda()
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM, group=group)
+    return float(t.item()), float(u.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# measured peaks and clocks
+# ---------------------------------------------------------------------------
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples (every 200 ms) while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# inputs
+# ---------------------------------------------------------------------------
+def make_matrix(fmt: int, K: int, N: int, seed: int, p0: float = 1.0 / 3.0):
+    """Packed weights (product codec), trits and alpha of one seeded matrix."""
+    import synth
+    import ternary_weight_03_b200 as tl
+    T = synth.trits(seed, N, K, p0=p0)
+    return tl.pack(fmt, T), T, synth.alpha_for(seed)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+class Sweep:
+    """Device-resident inputs of the GEMV sweep with rotating weight copies."""
+
+    def __init__(self, fmt: int, dev, shapes=SWEEP, ms=SWEEP_M, p0=1.0 / 3.0, seed0=0,
+                 min_rotation_bytes=3 * L2_BYTES):
+        import torch
+        import synth
+        import ternary_weight_03_b200 as tl
+        self.fmt, self.dev, self.ms = fmt, dev, ms
+        self.items = []  # (K, N, packed host, alpha, X per M)
+        per_set = 0
+        for i, (K, N) in enumerate(shapes):
+            P, _, alpha = make_matrix(fmt, K, N, seed0 + i, p0)
+            xs = {M: torch.from_numpy(synth.activations(seed0 + i, M, K)).to(dev) for M in ms}
+            self.items.append((K, N, P, alpha, xs))
+            per_set += P.nbytes
+        self.copies = max(2 * len(ms), -(-min_rotation_bytes // per_set))
+        self.dP = [[torch.from_numpy(P).to(dev) for (_, _, P, _, _) in self.items]
+                   for _ in range(self.copies)]
+        self.Y = {M: [torch.empty((M, N + (-N) % 8), dtype=torch.float16, device=dev)
+                      for (_, N, _, _, _) in self.items] for M in ms}
+        self.bytes_per_pass = sum(N * tl.row_bytes(fmt, K) for (K, N, _, _, _) in self.items)
+        self.bytes_per_step = self.bytes_per_pass * len(ms)
+        self.launches_per_step = len(self.items) * len(ms)
+        self.rotation_bytes = self.copies * per_set
+
+    def enqueue(self, step: int, stream, events=None):
+        """Enqueue the calls of one step on `stream` (optionally recording an
+        event after each call for per-launch timing)."""
+        import ternary_weight_03_b200 as tl
+        L = tl.lib()
+        s = stream.cuda_stream
+        j = 0
+        if events is not None:
+            events[0].record(stream)
+        for mi, M in enumerate(self.ms):
+            copy = (len(self.ms) * step + mi) % self.copies
+            for i, (K, N, _, alpha, xs) in enumerate(self.items):
+                dP, X, Y = self.dP[copy][i], xs[M], self.Y[M][i]
+                rc = L.tl_gemv(self.fmt, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(),
+                               X.stride(0), Y.data_ptr(), Y.stride(0), M, N, K, s)
+                if rc != 0:
+                    raise RuntimeError(f"tl_gemv -> {tl.status_str(rc)}")
+                j += 1
+                if events is not None:
+                    events[j].record(stream)
+
+
+def time_graphs(sweep: Sweep, steps: int, warmup: int, stream, clock_gpu: int | None = None):
+    """Capture one CUDA graph per rotation phase (event records between the
+    calls), warm up, then time `steps` replays with CUDA events.  Per-launch
+    kernel times come from the event records of the last timed replay of each
+    phase.  Returns (total ms, per-launch ms list, clocks summary)."""
+    import torch
+    nm = len(sweep.ms)
+    nphase = sweep.copies // nm if sweep.copies % nm == 0 else sweep.copies
+    graphs, evsets = [], []
+    with torch.cuda.stream(stream):
+        sweep.enqueue(0, stream)  # first call sets up per-device state outside capture
+        torch.cuda.synchronize()
+        for ph in range(nphase):
+            evs = [torch.cuda.Event(enable_timing=True, external=True)
+                   for _ in range(sweep.launches_per_step + 1)]
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                sweep.enqueue(ph, stream, evs)
+            graphs.append(g)
+            evsets.append(evs)
+    with torch.cuda.stream(stream):
+        for s in range(warmup):
+            graphs[s % nphase].replay()
+    torch.cuda.synchronize()
+    barrier()
+    sampler = ClockSampler(clock_gpu) if clock_gpu is not None else None
+    if sampler:
+        sampler.__enter__()
+    try:
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(stream):
+            start.record(stream)
+            for s in range(steps):
+                graphs[(warmup + s) % nphase].replay()
+            end.record(stream)
+        torch.cuda.synchronize()
+        total_ms = start.elapsed_time(end)
+    finally:
+        if sampler:
+            sampler.__exit__(None, None, None)
+    seen = sorted({(warmup + s) % nphase for s in range(steps)})
+    per_launch = [0.0] * sweep.launches_per_step
+    for ph in seen:
+        evs = evsets[ph]
+        for j in range(sweep.launches_per_step):
+            per_launch[j] += evs[j].elapsed_time(evs[j + 1]) / len(seen)
+    return total_ms, per_launch, (sampler.summary() if sampler else None)
+
+
+def time_e2e(sweep: Sweep, steps: int, warmup: int, stream):
+    """End to end through the C ABI from pinned host buffers: every step
+    copies its packed weights and activations host -> device, runs the twelve
+    calls and copies the outputs back.  Returns (ms, h2d bytes, d2h bytes)."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    L = tl.lib()
+    hP = [torch.from_numpy(P).pin_memory() for (_, _, P, _, _) in sweep.items]
+    hX = {M: [xs[M].cpu().pin_memory() for (_, _, _, _, xs) in sweep.items] for M in sweep.ms}
+    hY = {M: [torch.empty(tuple(y.shape), dtype=torch.float16).pin_memory() for y in sweep.Y[M]]
+          for M in sweep.ms}
+    dP = [torch.empty_like(p, device=sweep.dev) for p in hP]
+    dX = {M: [torch.empty_like(x, device=sweep.dev) for x in hX[M]] for M in sweep.ms}
+    h2d = sum(p.numel() for p in hP) * len(sweep.ms) + sum(
+        x.numel() * 2 for M in sweep.ms for x in hX[M])
+    d2h = sum(y.numel() * 2 for M in sweep.ms for y in hY[M])
+
+    def one_step():
+        for M in sweep.ms:
+            for i, (K, N, _, alpha, _) in enumerate(sweep.items):
+                dP[i].copy_(hP[i], non_blocking=True)
+                dX[M][i].copy_(hX[M][i], non_blocking=True)
+                Y = sweep.Y[M][i]
+                rc = L.tl_gemv(sweep.fmt, dP[i].data_ptr(), dP[i].stride(0), alpha,
+                               dX[M][i].data_ptr(), dX[M][i].stride(0), Y.data_ptr(), Y.stride(0),
+                               M, N, K, stream.cuda_stream)
+                if rc != 0:
+                    raise RuntimeError(f"tl_gemv -> {tl.status_str(rc)}")
+                hY[M][i].copy_(Y, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            one_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+    return a.elapsed_time(b), h2d, d2h
+
+
+def check_outputs(sweep: Sweep, samples: int = 64):
+    """Spot-check the last outputs of every call against the oracle."""
+    import oracle
+    import synth
+    o = oracle.get()
+    worst = 0.0
+    rng = np.random.default_rng(0)
+    for i, (K, N, P, alpha, xs) in enumerate(sweep.items):
+        T = synth.trits(i, N, K)
+        for M in sweep.ms:
+            X = xs[M].cpu().numpy()
+            Y = sweep.Y[M][i][:, :N].float().cpu().numpy().astype(np.float64)
+            ms = rng.integers(0, M, samples)
+            ns = rng.integers(0, N, samples)
+            ref = o.linear_at(T, X, alpha, ms, ns)
+            tol = oracle.tolerance(ref, X[ms], alpha)
+            err = np.abs(Y[ms, ns] - ref) / tol
+            if not (err <= 1.0).all():
+                raise AssertionError(f"bench output outside tolerance for shape {(K, N)} M={M}")
+            worst = max(worst, float(err.max()))
+    return worst
+
+
+def cpu_baseline(seconds: float = 10.0, threads: int | None = None):
+    """The oracle (unpack + double-precision layer) on a bounded sample of the
+    sweep: for every (shape, M), the first rows of the matrix, sized so the
+    whole sample takes about `seconds`.  Returns packed bytes/s and details."""
+    import oracle
+    import synth
+    o = oracle.get()
+    threads = threads or os.cpu_count() or 1
+    # calibrate on a small slice
+    K, N = SWEEP[0]
+    P, T, alpha = make_matrix(2, K, 64, 0)
+    X = synth.activations(0, 8, K)
+    t0 = time.perf_counter()
+    rc, Tu, _ = o.unpack(2, P, K)
+    o.linear(Tu, X, alpha, nthreads=threads)
+    per_trit_m = (time.perf_counter() - t0) / (64 * K * 8)
+    total_trit_m = sum(K * N for (K, N) in SWEEP) * sum(SWEEP_M)
+    frac = min(1.0, seconds / max(per_trit_m * total_trit_m, 1e-9))
+    done_bytes, elapsed, rows_used = 0, 0.0, []
+    for i, (K, N) in enumerate(SWEEP):
+        rows = max(threads, int(N * frac))
+        rows = min(rows, N)
+        Pm, Tm, alpha = make_matrix(2, K, rows, i)
+        for M in SWEEP_M:
+            X = synth.activations(i, M, K)
+            t0 = time.perf_counter()
+            rc, Tu, _ = o.unpack(2, Pm, K)
+            o.linear(Tu, X, alpha, nthreads=threads)
+            elapsed += time.perf_counter() - t0
+            done_bytes += rows * ((K + 3) // 4)
+        rows_used.append(rows)
+    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"first {rows_used} rows of each sweep matrix (both M), unpack + double "
+                      f"accumulation, {elapsed:.1f} s"}
+
+
+def secondary(dev, stream, quick: bool):
+    """1.6-bit sweep (p0 = 1/3), batched GEMM and the 30-layer decode step."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    out = {}
+    pk = peaks()
+    # 1.6-bit sweep
+    sw = Sweep(16, dev)
+    ms, per_launch, _ = time_graphs(sw, 5, 3, stream)
+    gbs = sw.bytes_per_step * 5 / (ms * 1e-3) / 1e9
+    out["gemv_1p6bit_sweep"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                                "ms_per_step": round(ms / 5, 4)}
+    del sw
+    torch.cuda.empty_cache()
+    # batched GEMM
+    gemm = {}
+    for (K, N) in ((4096, 14336), (14336, 4096)):
+        P, _, alpha = make_matrix(2, K, N, 0)
+        dP = torch.from_numpy(P).to(dev)
+        for M in ((16, 256, 4096) if quick else (16, 64, 256, 1024, 4096)):
+            import synth
+            X = torch.from_numpy(synth.activations(1, M, K)).to(dev)
+            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+            rc = tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
+                                  Y.data_ptr(), N, M, N, K, stream.cuda_stream)
+            if rc != 0:
+                gemm[f"M{M}_K{K}_N{N}"] = {"status": tl.status_str(rc)}
+                continue
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
+                                     Y.data_ptr(), N, M, N, K, stream.cuda_stream)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                a.record(stream)
+                for _ in range(reps):
+                    tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
+                                     Y.data_ptr(), N, M, N, K, stream.cuda_stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / reps
+            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+            gemm[f"M{M}_K{K}_N{N}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 1),
+                                       "frac_tensor": round(tf / pk["bf16_tflops"], 4)}
+    out["gemm_2bit"] = gemm
+    return out
+
+
+def run_gpu(args):
+    import torch
+    rank, local_rank, world = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    from ternary_weight_03_b200 import build
+    build.build()
+    import ternary_weight_03_b200 as tl
+    tl.lib()
+    stream = torch.cuda.Stream(device=dev)
+    pk = peaks()
+
+    sweep = Sweep(2, dev)
+    total_ms, per_launch, clocks = time_graphs(sweep, args.steps, args.warmup, stream,
+                                               clock_gpu=local_rank)
+    worst = check_outputs(sweep)
+    max_ms, total_bytes = reduce_step_time(total_ms, sweep.bytes_per_step * args.steps)
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    kernel_ms = sum(per_launch)
+    achieved = sweep.bytes_per_step / (kernel_ms * 1e-3) / 1e9
+    e2e_ms, h2d, d2h = time_e2e(sweep, max(1, min(args.steps, 5)), 1, stream)
+    e2e_steps = max(1, min(args.steps, 5))
+    e2e_max, e2e_bytes = reduce_step_time(e2e_ms, sweep.bytes_per_step * e2e_steps)
+    traffic = traffic_per_launch()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16 inputs, f32 accumulation",
+        "data": "synthetic (seeded SplitMix64 trits and N(0,1) fp16 activations)",
+        "config": {
+            "workload": WORKLOAD,
+            "packed_bytes_per_step": sweep.bytes_per_step,
+            "calls_per_step": sweep.launches_per_step,
+            "l2": f"inputs larger than L2: {sweep.copies} rotating copies of the packed "
+                  f"matrices ({sweep.rotation_bytes / 2**20:.0f} MiB) so every call reads HBM",
+            "timing": "CUDA graph per step, CUDA events on the launch stream",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "tlk::gemv_kernel<2>",
+            "achieved": round(achieved, 2),
+            "peak": pk["hbm_gbs"],
+            "unit": "GB/s",
+            "frac": round(achieved / pk["hbm_gbs"], 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": sweep.bytes_per_step // sweep.launches_per_step,
+            "avg_launch_us": round(kernel_ms * 1e3 / sweep.launches_per_step, 3),
+            "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({pk['source']})",
+        },
+        "e2e": {"value": round(e2e_bytes / (e2e_max * 1e-3) / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": sweep.launches_per_step * args.steps,
+        "clocks": clocks,
+        "max_err_over_tol": round(worst, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if not args.no_secondary:
+        line["secondary"] = secondary(dev, stream, quick=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def traffic_per_launch():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources (else None)."""
+    p = ROOT / "profiles" / "gemv2_sweep_traffic.json"
+    if not p.exists():
+        return None
+    try:
+        d = json.loads(p.read_text())
+        from ternary_weight_03_b200 import build
+        import hashlib
+        h = hashlib.sha256()
+        for f in sorted(build.DEPENDS):
+            h.update(Path(f).read_bytes())
+        if d.get("sources_sha256") != h.hexdigest():
+            return None
+        return d.get("dram_bytes_per_launch")
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    import synth
+    o = oracle.get()
+    threads = os.cpu_count() or 1
+    # each step: the first `rows` rows of every sweep matrix, both M, sized so
+    # that warmup + steps take about a minute in total
+    budget_s = 60.0 / max(1, args.steps + args.warmup)
+    K, N = SWEEP[0]
+    P, T, alpha = make_matrix(2, K, 64, 0)
+    X = synth.activations(0, 8, K)
+    t0 = time.perf_counter()
+    o.linear(o.unpack(2, P, K)[1], X, alpha, nthreads=threads)
+    per = (time.perf_counter() - t0) / (64 * K * 8)
+    frac = min(1.0, budget_s / max(per * sum(K * N for K, N in SWEEP) * sum(SWEEP_M), 1e-9))
+    mats = []
+    for i, (K, N) in enumerate(SWEEP):
+        rows = min(N, max(threads, int(N * frac)))
+        Pm, _, alpha = make_matrix(2, K, rows, i)
+        mats.append((K, rows, Pm, alpha, {M: synth.activations(i, M, K) for M in SWEEP_M}))
+    step_bytes = sum(rows * ((K + 3) // 4) for (K, rows, _, _, _) in mats) * len(SWEEP_M)
+
+    def step():
+        for (K, rows, Pm, alpha, xs) in mats:
+            for M in SWEEP_M:
+                o.linear(o.unpack(2, Pm, K)[1], xs[M], alpha, nthreads=threads)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    value = step_bytes * args.steps / el / 1e9
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el * 1e3 / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64 (oracle)", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "sample": f"first rows {[m[1] for m in mats]} of each "
+                   "matrix per step", "parallelism": "host threads"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"first rows {[m[1] for m in mats]} of each sweep matrix, "
+                                   "both M, per step"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_single(fmt: int, K: int, N: int, M: int, reps: int = 4):
+    """One seeded layer shape, `reps` calls through the C ABI (tl_gemv for
+    M <= 8, tl_gemm otherwise), nothing else on the device."""
+    import torch
+    import synth
+    import ternary_weight_03_b200 as tl
+    from ternary_weight_03_b200 import build
+    build.build()
+    P, _, alpha = make_matrix(fmt, K, N, 0)
+    dP = torch.from_numpy(P).cuda()
+    X = torch.from_numpy(synth.activations(1, M, K)).cuda()
+    for _ in range(reps):
+        Y = tl.linear(fmt, dP, alpha, X, K)
+    torch.cuda.synchronize()
+    print(json.dumps({"single": [fmt, K, N, M], "checksum": float(Y.float().abs().sum())}))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--single", metavar="FMT,K,N,M",
+                    help="run one seeded layer call 4 times and exit (for ncu captures)")
+    args = ap.parse_args(argv)
+    if args.single:
+        run_single(*[int(v) for v in args.single.split(",")])
+        return
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()
