@@ -9,6 +9,7 @@
 #include "tl_common.cuh"
 #include "tl_gemv.cuh"
 #include "tl_gemm.cuh"
+#include "tl_gemv_tc.cuh"
 
 namespace {
 
@@ -93,6 +94,9 @@ int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t
     const DeviceInfo *dev = device_info();
     if (!dev) return TL_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
+    if (fmt == TL_FMT_2BIT && tlk::gemv_tc_supported((int)N, (int)K))
+        return tlk::launch_gemv_tc(dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
+                                   dev->num_sms, s, &t_last_cuda_error);
     if (fmt == TL_FMT_2BIT) {
         const tlk::GemvShape sh = tlk::gemv_shape<2>((int)N, (int)K, dev->num_sms, gemv_occupancy);
         tlk::gemv_kernel<2><<<sh.grid, 32 * sh.warps, 0, s>>>(dT, ldp, alpha, dX, ldx, dY, ldy, M,

@@ -164,6 +164,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             decode2_exact(pw.y, a + 8);
             decode2_exact(pw.z, a + 16);
             decode2_exact(pw.w, a + 24);
+            // the packed bytes are consumed; order these generic reads before the
+            // TMA write that will refill this stage once the MMA releases it
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_after();
             tmem_st_32x32b_x32(tmem + lane_addr + gemm_acol_base(BN) + 32 * s, a);
             tc_wait_st();
