@@ -15,10 +15,11 @@
 //    memory, permuted so that it is the MMA B operand for the digit classes
 //    below (tokens m >= M are left undefined: their outputs are never stored);
 //  * eight decode warps (thread = weight row = TMEM lane) turn each 32-bit word
-//    of 16 digits into 8 fp16x2 registers with one LOP3 (or SHF+LOP3) each:
-//    digit d = t + 1 masked in place reads as the subnormal d * 2^(2c-24),
-//    c = 0..5 the digit's bit pair within its 16-bit half ("class"); the
-//    registers go to tensor memory with tcgen05.st as the MMA A operand;
+//    of 16 digits into 8 fp16x2 registers with one LOP3 each (plus one shift
+//    per word): digit d = t + 1 masked in place reads as the subnormal
+//    d * 2^(2c-24), c = 0..3 the digit's bit pair within its byte ("class");
+//    the registers go to a 3-slot ring in tensor memory with tcgen05.st as the
+//    MMA A operand;
 //  * one thread issues tcgen05.mma.kind::f16 (M = 128 rows, N = 16 tokens,
 //    K = 16), one fp32 accumulator per class, and recycles the A slots with
 //    tcgen05.commit;
@@ -41,17 +42,17 @@ constexpr int kTcStageRowBytes = 64;   // bytes per row per stage (256 trits)
 constexpr int kTcStages = 4;           // TMA ring depth
 constexpr int kTcThreads = 320;        // warp 0 TMA, warp 1 MMA, warps 2..9 decode
 constexpr int kTcMaxStagesPerCta = 8;  // K range per CTA <= 2048 trits
-constexpr int kTcTmemCols = 256;       // 6 class accumulators x 16 + 2 A slots x 64
+constexpr int kTcTmemCols = 256;       // 4 class accumulators x 16 + 3 A slots x 64
 constexpr int kTcAccCol = 0;           // class c accumulator at columns [16c, 16c + 16)
-constexpr int kTcSlotCol = 128;        // A slot h at [128 + 64h, 128 + 64h + 64)
+constexpr int kTcSlotCol = 64;         // A slot i at [64 + 64i, 64 + 64i + 64)
+constexpr int kTcSlots = 3;
 constexpr int kTcBlockBytes = 4096;    // permuted activations per 128-trit block (8 x 512)
 constexpr int kTcMaxCluster = 8;
 
-// class-part ci (0..7): digit shift s' within the 16-bit half, accumulator class
-__host__ __device__ constexpr int tc_shift(int ci) {
-    return ci == 0 ? 0 : ci == 1 ? 6 : ci == 2 ? 1 : ci == 3 ? 7 : ci - 2;
-}
-__host__ __device__ constexpr int tc_class(int ci) { return ci < 2 ? 0 : ci < 4 ? 1 : ci - 2; }
+// class-part ci (0..7) holds digits (ci, 8 + ci) of a word; its bit pair
+// within the byte, and so its accumulator class, is ci & 3.
+__host__ __device__ constexpr int tc_shift(int ci) { return ci; }
+__host__ __device__ constexpr int tc_class(int ci) { return ci & 3; }
 
 struct TcSmem {
     static constexpr uint32_t wstage_bytes = 128u * kTcStageRowBytes;  // 8 KB
@@ -117,17 +118,19 @@ __device__ __forceinline__ void tmem_st_32x32b_x64(uint32_t taddr, const uint32_
 }
 
 // Class-masked registers of one 32-bit word (16 digits, digit i at bits 2i):
-// register ci holds digits (s', 8 + s') of the word, s' = tc_shift(ci).
+// register ci holds digits (ci, 8 + ci) of the word in its low / high half,
+// at bit pair ci & 3 of the half's low byte (digits 4..7 and 12..15 come from
+// the word shifted right by 8).
 __device__ __forceinline__ void tc_decode_word(uint32_t w, uint32_t *r8 /* stride 8 */) {
-    const uint32_t h = w >> 12;
-    r8[0 * 8] = w & 0x00030003u;  // s'=0, class 0
-    r8[1 * 8] = h & 0x00030003u;  // s'=6, class 0
-    r8[2 * 8] = w & 0x000C000Cu;  // s'=1, class 1
-    r8[3 * 8] = h & 0x000C000Cu;  // s'=7, class 1
-    r8[4 * 8] = w & 0x00300030u;  // s'=2, class 2
-    r8[5 * 8] = w & 0x00C000C0u;  // s'=3, class 3
-    r8[6 * 8] = w & 0x03000300u;  // s'=4, class 4
-    r8[7 * 8] = w & 0x0C000C00u;  // s'=5, class 5 (exponent bits: 2^(d-15) = d * 2^-14)
+    const uint32_t h = w >> 8;
+    r8[0 * 8] = w & 0x00030003u;  // digits 0, 8   class 0
+    r8[1 * 8] = w & 0x000C000Cu;  // digits 1, 9   class 1
+    r8[2 * 8] = w & 0x00300030u;  // digits 2, 10  class 2
+    r8[3 * 8] = w & 0x00C000C0u;  // digits 3, 11  class 3
+    r8[4 * 8] = h & 0x00030003u;  // digits 4, 12  class 0
+    r8[5 * 8] = h & 0x000C000Cu;  // digits 5, 13  class 1
+    r8[6 * 8] = h & 0x00300030u;  // digits 6, 14  class 2
+    r8[7 * 8] = h & 0x00C000C0u;  // digits 7, 15  class 3
 }
 
 __global__ void __launch_bounds__(kTcThreads, 2)
@@ -142,9 +145,9 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TcSmem::bar_off);
     uint64_t *wfull = bars;                   // [kTcStages] TMA -> decoders
     uint64_t *wempty = wfull + kTcStages;     // [kTcStages] decoders -> TMA
-    uint64_t *afull = wempty + kTcStages;     // [2] decode set h -> MMA
-    uint64_t *aempty = afull + 2;             // [2] MMA commit -> decode set h
-    uint64_t *done = aempty + 2;              // last MMA committed -> epilogue
+    uint64_t *afull = wempty + kTcStages;     // [kTcSlots] decoders -> MMA
+    uint64_t *aempty = afull + kTcSlots;      // [kTcSlots] MMA commit -> decoders
+    uint64_t *done = aempty + kTcSlots;       // last MMA committed -> epilogue
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -164,9 +167,9 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
             mbar_init(&wfull[s], 1);
             mbar_init(&wempty[s], 256);
         }
-        for (int h = 0; h < 2; ++h) {
-            mbar_init(&afull[h], 128);
-            mbar_init(&aempty[h], 1);
+        for (int i = 0; i < kTcSlots; ++i) {
+            mbar_init(&afull[i], 128);
+            mbar_init(&aempty[i], 1);
         }
         mbar_init(done, 1);
         fence_mbar_init();
@@ -252,19 +255,19 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
             constexpr uint32_t idesc = idesc_f16_f32(128, 16);
             const uint32_t xbase = smem_u32(xperm);
             for (int lb = 0; lb < nblk; ++lb) {
-                const int h = lb & 1;
-                if (!mbar_wait(&afull[h], (lb >> 1) & 1)) break;
+                const int slot = lb % kTcSlots;
+                if (!mbar_wait(&afull[slot], (lb / kTcSlots) & 1)) break;
                 tc_fence_after();
 #pragma unroll
                 for (int ci = 0; ci < 8; ++ci) {
                     const uint64_t bdesc =
                         sdesc_kinter(xbase + (uint32_t)(lb * 8 + ci) * 512u, 128u, 256u);
                     const uint32_t acc = tmem + kTcAccCol + 16 * tc_class(ci);
-                    const uint32_t a = tmem + kTcSlotCol + 64 * h + 8 * ci;
-                    const bool first = lb == 0 && (ci == 0 || ci == 2 || ci >= 4);
+                    const uint32_t a = tmem + kTcSlotCol + 64 * slot + 8 * ci;
+                    const bool first = lb == 0 && ci < 4;
                     tc_mma_ts(acc, a, bdesc, idesc, first ? 0u : 1u);
                 }
-                tc_commit(&aempty[h]);
+                tc_commit(&aempty[slot]);
             }
             tc_commit(done);
         }
@@ -288,7 +291,9 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
                 c1 = c0;
             }
             const int lb = 2 * st + h;
-            if (lb >= 2 && !(ok = mbar_wait(&aempty[h], ((lb >> 1) - 1) & 1))) break;
+            const int slot = lb % kTcSlots;
+            if (lb >= kTcSlots && !(ok = mbar_wait(&aempty[slot], ((lb / kTcSlots) - 1) & 1)))
+                break;
             tc_fence_after();
             uint32_t a[64];
             tc_decode_word(c0.x, a + 0);
@@ -303,10 +308,10 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
             // proxy fence orders these generic reads before the next TMA write
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(&wempty[s]);
-            tmem_st_32x32b_x64(tmem + lane_addr + kTcSlotCol + 64 * h, a);
+            tmem_st_32x32b_x64(tmem + lane_addr + kTcSlotCol + 64 * slot, a);
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&afull[h]);
+            mbar_arrive(&afull[slot]);
         }
         // ---- epilogue part 1: combine classes, partial sums to shared memory ----
         if (h == 0) {
@@ -317,7 +322,7 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
             if (ok && nblk > 0) {
                 tc_fence_after();
 #pragma unroll
-                for (int part = 0; part < 3; ++part) {
+                for (int part = 0; part < 2; ++part) {
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tmem + lane_addr + kTcAccCol + 32 * part, v);
                     tc_wait_ld();
@@ -325,8 +330,7 @@ gemv2_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__re
                     for (int i = 0; i < 32; ++i) {
                         const int cls = 2 * part + (i >> 4);  // columns 16 c + m
                         const float scale = cls == 0 ? 16777216.f : cls == 1 ? 4194304.f
-                                          : cls == 2 ? 1048576.f : cls == 3 ? 262144.f
-                                          : cls == 4 ? 65536.f : 16384.f;
+                                          : cls == 2 ? 1048576.f : 262144.f;
                         s16[i & 15] += __uint_as_float(v[i]) * scale;
                     }
                 }
