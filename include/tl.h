@@ -115,6 +115,22 @@ int tl_unpack(int fmt, const uint8_t *P, int64_t N, int64_t K, int64_t ldp, int8
 int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
             int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream);
 
+/* Flags of tl_gemv_ex. */
+#define TL_FLAG_PDL 1u /* programmatic dependent launch, see tl_gemv_ex */
+
+/* tl_gemv with launch flags (tl_gemv is tl_gemv_ex with flags = 0).
+ * TL_FLAG_PDL: the kernel is launched with programmatic stream
+ * serialization, so it may begin while the preceding kernel on `stream` is
+ * still running.  Before it waits for that kernel it only streams the packed
+ * weights dT; it reads X and writes Y after the preceding work has completed
+ * and its memory is visible.  The caller therefore promises that dT is not
+ * written by any work still in flight on the stream (true of static layer
+ * weights).  Works inside CUDA-graph capture.  Other flag bits:
+ * TL_ERR_INVALID_ARG. */
+int tl_gemv_ex(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+               int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K,
+               unsigned int flags, void *stream);
+
 /* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and
  * rules as tl_gemv (tensor-core kernel: packed tiles are expanded to fp16
  * on chip and multiplied with tcgen05 MMAs accumulating in fp32). */

@@ -36,6 +36,8 @@ SIGNATURES = {
     "tl_pack16": (_i32, [_p, _i64, _i64, _i64, _p, _i64]),
     "tl_unpack": (_i32, [_i32, _p, _i64, _i64, _i64, _p, _i64, ctypes.POINTER(_i64)]),
     "tl_gemv": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _p]),
+    "tl_gemv_ex": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64,
+                          ctypes.c_uint, _p]),
     "tl_gemm": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _p]),
     "tl_device_status": (_i32, [_p]),
 }
@@ -126,7 +128,11 @@ def _stream_ptr(stream) -> int:
     return int(stream.cuda_stream)
 
 
-def _layer(fn_name: str, fmt: int, dT, alpha: float, X, K: int, out=None, stream=None, M=None):
+FLAG_PDL = 1
+
+
+def _layer(fn_name: str, fmt: int, dT, alpha: float, X, K: int, out=None, stream=None, M=None,
+           flags=None):
     import torch
     assert dT.is_cuda and dT.dtype == torch.uint8 and dT.dim() == 2
     assert X.is_cuda and X.dtype == torch.float16 and X.dim() == 2
@@ -135,15 +141,20 @@ def _layer(fn_name: str, fmt: int, dT, alpha: float, X, K: int, out=None, stream
     if out is None:
         out = torch.empty((M, N + (-N) % 8), dtype=torch.float16, device=X.device)
     assert out.is_cuda and out.dtype == torch.float16
-    rc = getattr(lib(), fn_name)(fmt, dT.data_ptr(), dT.stride(0), float(alpha), X.data_ptr(),
-                                 X.stride(0), out.data_ptr(), out.stride(0), M, N, K,
-                                 _stream_ptr(stream))
+    args = [fmt, dT.data_ptr(), dT.stride(0), float(alpha), X.data_ptr(), X.stride(0),
+            out.data_ptr(), out.stride(0), M, N, K]
+    if flags is not None:
+        args.append(int(flags))
+    rc = getattr(lib(), fn_name)(*args, _stream_ptr(stream))
     _check(fn_name, rc)
     return out[:, :N]
 
 
-def gemv(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None):
-    """Y[M, N] = alpha * X T^T for 1 <= M <= 8 (decode-shaped)."""
+def gemv(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None, flags: int = 0):
+    """Y[M, N] = alpha * X T^T for 1 <= M <= 8 (decode-shaped).  flags=FLAG_PDL:
+    programmatic dependent launch (dT must not be written by in-flight work)."""
+    if flags:
+        return _layer("tl_gemv_ex", fmt, dT, alpha, X, K, out, stream, flags=flags)
     return _layer("tl_gemv", fmt, dT, alpha, X, K, out, stream)
 
 

@@ -47,6 +47,17 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Programmatic dependent launch.  wait: block until the preceding grid on the
+// stream has completed and its memory is visible (a no-op when the kernel was
+// launched without the programmatic-serialization attribute).  launch:
+// allow the next grid on the stream to begin its own pre-wait prologue.
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint16_t f32_to_f16_bits(float v) {
     return __half_as_ushort(__float2half_rn(v));
 }

@@ -9,7 +9,7 @@
 #include "tl_common.cuh"
 #include "tl_gemv.cuh"
 #include "tl_gemm.cuh"
-#include "tl_gemv_tc.cuh"
+#include "tl_gemv3.cuh"
 
 namespace {
 
@@ -86,29 +86,53 @@ extern "C" {
 
 int tl_last_cuda_error(void) { return t_last_cuda_error; }
 
-int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
-            int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream) {
+int tl_gemv_ex(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+               int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K,
+               unsigned int flags, void *stream) {
     if (M < 1 || M > TL_GEMV_MAX_M) return TL_ERR_INVALID_ARG;
+    if (flags & ~(unsigned int)TL_FLAG_PDL) return TL_ERR_INVALID_ARG;
     int rc = check_layer_args(fmt, dT, ldp, dX, ldx, dY, ldy, N, K);
     if (rc != TL_OK) return rc;
     const DeviceInfo *dev = device_info();
     if (!dev) return TL_ERR_CUDA;
     cudaStream_t s = (cudaStream_t)stream;
-    if (fmt == TL_FMT_2BIT && tlk::gemv_tc_supported((int)N, (int)K))
-        return tlk::launch_gemv_tc(dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
-                                   dev->num_sms, s, &t_last_cuda_error);
+    const bool pdl = (flags & TL_FLAG_PDL) != 0;
+    if (fmt == TL_FMT_2BIT && tlk::gemv3_supported<2>((int)K))
+        return tlk::launch_gemv3<2>(dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
+                                    dev->num_sms, pdl, s, &t_last_cuda_error);
+    if (fmt == TL_FMT_1P6BIT && tlk::gemv3_supported<16>((int)K))
+        return tlk::launch_gemv3<16>(dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
+                                     dev->num_sms, pdl, s, &t_last_cuda_error);
+    // K beyond what one cluster can stage: the register-streaming kernel
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.stream = s;
+    cudaError_t e;
     if (fmt == TL_FMT_2BIT) {
         const tlk::GemvShape sh = tlk::gemv_shape<2>((int)N, (int)K, dev->num_sms, gemv_occupancy);
-        tlk::gemv_kernel<2><<<sh.grid, 32 * sh.warps, 0, s>>>(dT, ldp, alpha, dX, ldx, dY, ldy, M,
-                                                             (int)N, (int)K, sh.tiles_per_cta);
+        cfg.gridDim = dim3((unsigned)sh.grid);
+        cfg.blockDim = dim3((unsigned)(32 * sh.warps));
+        e = cudaLaunchKernelEx(&cfg, tlk::gemv_kernel<2>, dT, ldp, alpha, dX, ldx, dY, ldy, M,
+                               (int)N, (int)K, sh.tiles_per_cta);
     } else {
         const tlk::GemvShape sh = tlk::gemv_shape<16>((int)N, (int)K, dev->num_sms, gemv_occupancy);
-        tlk::gemv_kernel<16><<<sh.grid, 32 * sh.warps, 0, s>>>(dT, ldp, alpha, dX, ldx, dY, ldy, M,
-                                                              (int)N, (int)K, sh.tiles_per_cta);
+        cfg.gridDim = dim3((unsigned)sh.grid);
+        cfg.blockDim = dim3((unsigned)(32 * sh.warps));
+        e = cudaLaunchKernelEx(&cfg, tlk::gemv_kernel<16>, dT, ldp, alpha, dX, ldx, dY, ldy, M,
+                               (int)N, (int)K, sh.tiles_per_cta);
     }
-    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
     return TL_OK;
+}
+
+int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+            int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream) {
+    return tl_gemv_ex(fmt, dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, 0u, stream);
 }
 
 int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,

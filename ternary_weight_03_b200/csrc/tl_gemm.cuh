@@ -205,20 +205,6 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 }
 
 // ---- host side ---------------------------------------------------------------
-inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
 inline size_t gemm_smem_bytes(int bn) {
     return 1024 + kGemmStages * ((size_t)bn * 128 + kGemmRows * 16) + (3 * kGemmStages + 1) * 8 +
            16;

@@ -259,6 +259,11 @@ gemv_kernel(const uint8_t *__restrict__ P, int64_t ldp, float alpha, const uint1
                 rb[i] = ld_stream(pB + (int64_t)(kg_begin + i) * strideB);
             }
         }
+        if (it == 0) {
+            // weights requested; activations and outputs may belong to preceding work
+            pdl_launch_dependents();
+            pdl_wait();
+        }
         for (int base = kg_begin; base < kmain; base += kGemvDepth) {
 #pragma unroll
             for (int i = 0; i < kGemvDepth; ++i) {

@@ -76,3 +76,11 @@ def test_gemm_argument_rules(L):
 def test_build_flags_target_sm100a():
     flags = " ".join(tlbuild.NVCC_FLAGS)
     assert "arch=compute_100a,code=sm_100a" in flags and "-lineinfo" in flags
+
+
+def test_gemv_ex_flags(L):
+    assert gemv_rc(L, fn="tl_gemv", M=0) == 1
+    A_ = 0x10000
+    # unknown flag bits are rejected before anything reaches a device
+    assert L.tl_gemv_ex(2, A_, 256, 1.0, A_, 1024, A_, 1024, 1, 1024, 1024, 2, None) == 1
+    assert L.tl_gemv_ex(2, A_, 256, 1.0, A_, 1024, A_, 1024, 9, 1024, 1024, 1, None) == 1
