@@ -548,7 +548,7 @@ def run_gpu(args):
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "tlk::gemv2_tc_kernel",
+            "kernel": "tlk::gemv3_kernel<2>",
             "achieved": round(achieved, 2),
             "peak": pk["hbm_gbs"],
             "unit": "GB/s",

@@ -198,6 +198,20 @@ __device__ __forceinline__ void st_dsmem_f32(uint32_t local_addr, uint32_t rank,
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
 }
+// Store two floats into CTA `rank`'s shared memory at the address that is
+// `local_addr` in this CTA, completing `bytes` on that CTA's mbarrier at
+// `local_bar` (also mapped to `rank`).
+__device__ __forceinline__ void st_async_v2_f32(uint32_t local_addr, uint32_t rank,
+                                                uint32_t local_bar, float a, float b) {
+    uint32_t raddr, rbar;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(local_addr), "r"(rank));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rbar) : "r"(local_bar), "r"(rank));
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
+            raddr),
+        "f"(a), "f"(b), "r"(rbar)
+        : "memory");
+}
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {
     uint32_t remote;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
