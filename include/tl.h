@@ -38,6 +38,7 @@
 #ifndef TERNARY_TL_H
 #define TERNARY_TL_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -130,6 +131,74 @@ int tl_gemv(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t
 int tl_gemv_ex(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
                int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K,
                unsigned int flags, void *stream);
+
+/* ---- a batch of decode-shaped layers in one launch ---------------------- */
+
+#define TL_GEMV_BATCH_MAX 4096    /* layers per batch */
+#define TL_LAYER_READS_EARLIER 1u /* tl_gemv_layer.flags, see tl_gemv_batch_plan */
+
+/* One layer of a batch: the arguments of tl_gemv for that layer. */
+typedef struct tl_gemv_layer {
+    const uint8_t *dT;   /* packed T, N rows of ldp bytes (device) */
+    int64_t ldp;
+    float alpha;
+    const uint16_t *dX;  /* M x K binary16 activations, row stride ldx (device) */
+    int64_t ldx;
+    uint16_t *dY;        /* M x N binary16 outputs, row stride ldy (device) */
+    int64_t ldy;
+    int M;               /* 1 .. TL_GEMV_MAX_M */
+    int64_t N, K;
+    unsigned int flags;  /* 0 or TL_LAYER_READS_EARLIER */
+} tl_gemv_layer;
+
+/* A planned batch: filled by tl_gemv_batch_plan, read by tl_gemv_batch_run.
+ * Plain data owned by the caller; treat the fields as read-only. */
+typedef struct tl_gemv_plan {
+    int fmt, count, max_m, total_items, total_tiles;
+    void *dWorkspace;
+    size_t workspace_bytes;
+} tl_gemv_plan;
+
+/* Workspace bytes a batch needs: the layer table and one TMA descriptor per
+ * layer (~200 B per layer), counters, and fp32 partial sums of the layers
+ * whose rows are split across CTAs (about N * M * 4 * K / 2048 bytes per
+ * such layer).  Validates the batch like tl_gemv_batch_plan.  Pure host
+ * function. */
+int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes);
+
+/* Plans count (1 .. TL_GEMV_BATCH_MAX) decode-shaped layers of one format
+ * for single-launch execution by tl_gemv_batch_run.  Every layer follows the
+ * argument rules of tl_gemv; layers[] is host memory, read before the call
+ * returns.  Writes the layer table and the layers' TMA descriptors into
+ * dWorkspace (device memory of at least tl_gemv_batch_bytes() bytes,
+ * 256-byte aligned, owned by the caller) and zeroes its counters, with
+ * blocking copies: the call synchronizes the device and may not be captured
+ * into a CUDA graph.  Plan once, run many times; the plan holds the
+ * pointers of T, X and Y, so a batch on other buffers needs a new plan.
+ * Dependencies: a layer with TL_LAYER_READS_EARLIER (not allowed on layer
+ * 0) reads its X only after every earlier layer of the batch has stored its
+ * Y, so it may consume their outputs (a chain of layers); without the flag,
+ * X must not be written by any layer of the batch.  No Y may overlap another
+ * layer's Y, X or T.  Errors: TL_ERR_INVALID_ARG (bad layer, count or
+ * workspace too small), TL_ERR_ALIGN, TL_ERR_CUDA. */
+int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dWorkspace,
+                       size_t workspace_bytes, tl_gemv_plan *plan);
+
+/* Runs a planned batch in ONE persistent launch: every layer computes
+ * exactly what tl_gemv computes.  The launch streams the packed weights of
+ * all layers back to back ("What carries the argument": decoding is bound by
+ * memory bandwidth), splitting long rows across CTAs; split rows are summed
+ * in a fixed order, so results are deterministic.  Each launch that
+ * completes leaves the workspace counters at zero, so the plan can be run
+ * again without clearing; after a launch that ends in TL_ERR_TIMEOUT
+ * (tl_device_status) plan again.  Launches of one plan (one workspace) must
+ * be ordered on one stream.  flags: 0 or TL_FLAG_PDL (as for tl_gemv_ex:
+ * the first weights are fetched while the preceding kernel finishes; X, Y
+ * and the workspace counters are touched only after it completed).
+ * Asynchronous, allocates nothing, may be captured into a CUDA graph.
+ * Errors: TL_ERR_INVALID_ARG (plan not filled by tl_gemv_batch_plan, bad
+ * flags), TL_ERR_CUDA. */
+int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream);
 
 /* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and
  * rules as tl_gemv (tensor-core kernel: packed tiles are expanded to fp16

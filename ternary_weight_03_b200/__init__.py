@@ -2,7 +2,7 @@
 
 Every step of the layer runs inside ``libternary.so``: the host codec
 (tl_pack2 / tl_pack16 / tl_unpack) and the sm_100a kernels (tl_gemv,
-tl_gemm).  PyTorch is used only for device buffers and streams.  There is no
+tl_gemm, tl_gemv_batch).  PyTorch is used only for device buffers and streams.  There is no
 fallback: if the library is missing or a call fails, an exception is raised.
 
 Functions take numpy arrays (host codec) or torch CUDA tensors (layer calls).
@@ -26,6 +26,25 @@ GEMM_MIN_M = 16
 STATUS = {0: "TL_OK", 1: "TL_ERR_INVALID_ARG", 2: "TL_ERR_BAD_TRIT", 3: "TL_ERR_BAD_CODE",
           4: "TL_ERR_ALIGN", 5: "TL_ERR_CUDA", 6: "TL_ERR_TIMEOUT", 7: "TL_ERR_UNSUPPORTED"}
 
+GEMV_BATCH_MAX = 4096
+LAYER_READS_EARLIER = 1
+
+
+class Layer(ctypes.Structure):
+    """tl_gemv_layer: one layer of a tl_gemv_batch call (device pointers)."""
+    _fields_ = [("dT", ctypes.c_void_p), ("ldp", ctypes.c_int64), ("alpha", ctypes.c_float),
+                ("dX", ctypes.c_void_p), ("ldx", ctypes.c_int64), ("dY", ctypes.c_void_p),
+                ("ldy", ctypes.c_int64), ("M", ctypes.c_int), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("flags", ctypes.c_uint)]
+
+
+class Plan(ctypes.Structure):
+    """tl_gemv_plan: a planned batch (filled by tl_gemv_batch_plan)."""
+    _fields_ = [("fmt", ctypes.c_int), ("count", ctypes.c_int), ("max_m", ctypes.c_int),
+                ("total_items", ctypes.c_int), ("total_tiles", ctypes.c_int),
+                ("dWorkspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+
+
 # (name, restype, argtypes) of every symbol the C header declares
 _i64, _i32, _p, _f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_float
 SIGNATURES = {
@@ -39,6 +58,11 @@ SIGNATURES = {
     "tl_gemv_ex": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64,
                           ctypes.c_uint, _p]),
     "tl_gemm": (_i32, [_i32, _p, _i64, _f32, _p, _i64, _p, _i64, _i32, _i64, _i64, _p]),
+    "tl_gemv_batch_bytes": (_i32, [_i32, _i32, ctypes.POINTER(Layer),
+                                   ctypes.POINTER(ctypes.c_size_t)]),
+    "tl_gemv_batch_plan": (_i32, [_i32, _i32, ctypes.POINTER(Layer), _p, ctypes.c_size_t,
+                                  ctypes.POINTER(Plan)]),
+    "tl_gemv_batch_run": (_i32, [ctypes.POINTER(Plan), ctypes.c_uint, _p]),
     "tl_device_status": (_i32, [_p]),
 }
 
@@ -178,6 +202,46 @@ def linear(fmt: int, dT, alpha: float, X, K: int, out=None, stream=None):
         gemv(fmt, dT, alpha, X[GEMV_MAX_M:], K, out[GEMV_MAX_M:], stream)
         return out[:, :N]
     return gemm(fmt, dT, alpha, X, K, out, stream)
+
+
+def make_layers(fmt: int, specs) -> ctypes.Array:
+    """ctypes array of tl_gemv_layer from (dT, alpha, X, K, Y[, flags]) tuples of
+    torch CUDA tensors (dT uint8 [N, ldp]; X, Y fp16 with M rows)."""
+    import torch
+    arr = (Layer * len(specs))()
+    for i, sp in enumerate(specs):
+        dT, alpha, X, K, Y = sp[:5]
+        flags = sp[5] if len(sp) > 5 else 0
+        assert dT.is_cuda and dT.dtype == torch.uint8 and dT.dim() == 2
+        assert X.is_cuda and X.dtype == torch.float16 and Y.dtype == torch.float16
+        arr[i] = Layer(dT.data_ptr(), dT.stride(0), float(alpha), X.data_ptr(), X.stride(0),
+                       Y.data_ptr(), Y.stride(0), X.shape[0], dT.shape[0], int(K), int(flags))
+    return arr
+
+
+def gemv_batch_bytes(fmt: int, layers) -> int:
+    """Workspace bytes of a batch (a ctypes layer array from make_layers)."""
+    n = ctypes.c_size_t(0)
+    _check("tl_gemv_batch_bytes", lib().tl_gemv_batch_bytes(fmt, len(layers), layers,
+                                                              ctypes.byref(n)))
+    return int(n.value)
+
+
+def gemv_batch_plan(fmt: int, layers, workspace) -> Plan:
+    """Plan a batch into `workspace` (a CUDA uint8 tensor, 256-byte aligned, of
+    at least gemv_batch_bytes bytes, kept alive by the caller).  Blocking."""
+    plan = Plan()
+    _check("tl_gemv_batch_plan",
+           lib().tl_gemv_batch_plan(fmt, len(layers), layers, workspace.data_ptr(),
+                                    workspace.numel() * workspace.element_size(),
+                                    ctypes.byref(plan)))
+    return plan
+
+
+def gemv_batch_run(plan: Plan, stream=None, flags: int = 0):
+    """Run a planned batch in one launch (asynchronous, graph-capturable)."""
+    _check("tl_gemv_batch_run", lib().tl_gemv_batch_run(ctypes.byref(plan), int(flags),
+                                                          _stream_ptr(stream)))
 
 
 def device_status(stream=None) -> int:

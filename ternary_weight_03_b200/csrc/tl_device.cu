@@ -1,8 +1,9 @@
 // tl_device.cu -- device entry points of libternary: argument validation,
-// kernel selection and launch for tl_gemv / tl_gemm, and the device error
-// word behind tl_device_status.
+// kernel selection and launch for tl_gemv / tl_gemm / tl_gemv_batch, and the
+// device error word behind tl_device_status.
 #include <cstdint>
 #include <mutex>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "tl.h"
@@ -10,6 +11,7 @@
 #include "tl_gemv.cuh"
 #include "tl_gemm.cuh"
 #include "tl_gemv3.cuh"
+#include "tl_gemvp.cuh"
 
 namespace {
 
@@ -80,6 +82,28 @@ int check_layer_args(int fmt, const uint8_t *dT, int64_t ldp, const uint16_t *dX
     return TL_OK;
 }
 
+// Validates a batch and converts it into the persistent kernel's host layers.
+int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::GpHostLayer *out) {
+    if (fmt != TL_FMT_2BIT && fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
+    if (count < 1 || count > TL_GEMV_BATCH_MAX || !layers) return TL_ERR_INVALID_ARG;
+    int64_t items = 0;
+    for (int l = 0; l < count; ++l) {
+        const tl_gemv_layer &a = layers[l];
+        if (a.M < 1 || a.M > TL_GEMV_MAX_M) return TL_ERR_INVALID_ARG;
+        if (a.flags & ~(unsigned int)TL_LAYER_READS_EARLIER) return TL_ERR_INVALID_ARG;
+        if (l == 0 && (a.flags & TL_LAYER_READS_EARLIER)) return TL_ERR_INVALID_ARG;
+        int rc = check_layer_args(fmt, a.dT, a.ldp, a.dX, a.ldx, a.dY, a.ldy, a.N, a.K);
+        if (rc != TL_OK) return rc;
+        if (a.ldx > INT32_MAX || a.ldy > INT32_MAX) return TL_ERR_INVALID_ARG;
+        const int64_t groups = (tl_packed_row_bytes(fmt, a.K) + 63) / 64;
+        items += ((a.N + tlk::kGpRows - 1) / tlk::kGpRows) * groups;  // upper bound
+        if (items > INT32_MAX / 2) return TL_ERR_INVALID_ARG;
+        out[l] = tlk::GpHostLayer{a.dT, a.dX, a.dY, a.ldp, a.ldx, a.ldy, a.alpha, a.M, (int)a.N,
+                                  (int)a.K, (a.flags & TL_LAYER_READS_EARLIER) != 0};
+    }
+    return TL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -142,6 +166,71 @@ int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t
     if (rc != TL_OK) return rc;
     return tlk::launch_gemm(fmt, dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
                             (cudaStream_t)stream, &t_last_cuda_error);
+}
+
+int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes) {
+    if (!bytes) return TL_ERR_INVALID_ARG;
+    std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
+    int rc = batch_layers(fmt, count, layers, h.data());
+    if (rc != TL_OK) return rc;
+    std::vector<tlk::GpLayer> table(count);
+    *bytes = tlk::gp_schedule(fmt, count, h.data(), table.data()).bytes;
+    return TL_OK;
+}
+
+int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dWorkspace,
+                       size_t workspace_bytes, tl_gemv_plan *plan) {
+    if (!plan || !dWorkspace) return TL_ERR_INVALID_ARG;
+    if (((uintptr_t)dWorkspace & 255u) != 0) return TL_ERR_ALIGN;
+    std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
+    int rc = batch_layers(fmt, count, layers, h.data());
+    if (rc != TL_OK) return rc;
+    std::vector<tlk::GpLayer> table(count);
+    const tlk::GpSchedule sc = tlk::gp_schedule(fmt, count, h.data(), table.data());
+    if (sc.bytes > workspace_bytes) return TL_ERR_INVALID_ARG;
+    std::vector<CUtensorMap> maps(count);
+    for (int l = 0; l < count; ++l)
+        if (!tlk::gp_encode_map(fmt, h[l], &maps[l])) return TL_ERR_CUDA;
+    if (!device_info()) return TL_ERR_CUDA;
+    const tlk::GpWsLayout wl(count, sc.total_tiles, sc.floats);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(dWorkspace);
+    cudaError_t e = cudaMemset(ws, 0, wl.layers);  // counters
+    if (e == cudaSuccess)
+        e = cudaMemcpy(ws + wl.layers, table.data(), sizeof(tlk::GpLayer) * count,
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(ws + wl.maps, maps.data(), sizeof(CUtensorMap) * count,
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(ws + wl.tiles, 0, (size_t)sc.total_tiles * 4u);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    plan->fmt = fmt;
+    plan->count = count;
+    plan->max_m = sc.maxM;
+    plan->total_items = sc.total_items;
+    plan->total_tiles = sc.total_tiles;
+    plan->dWorkspace = dWorkspace;
+    plan->workspace_bytes = workspace_bytes;
+    return TL_OK;
+}
+
+int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream) {
+    if (!plan || !plan->dWorkspace) return TL_ERR_INVALID_ARG;
+    if (flags & ~(unsigned int)TL_FLAG_PDL) return TL_ERR_INVALID_ARG;
+    if (plan->fmt != TL_FMT_2BIT && plan->fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
+    if (plan->count < 1 || plan->count > TL_GEMV_BATCH_MAX || plan->max_m < 1 ||
+        plan->max_m > TL_GEMV_MAX_M || plan->total_items < 1 || plan->total_tiles < 1)
+        return TL_ERR_INVALID_ARG;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return TL_ERR_CUDA;
+    const tlk::GpArgs a = tlk::gp_args(plan->dWorkspace, plan->count, plan->total_items,
+                                       plan->total_tiles, plan->max_m);
+    const bool pdl = (flags & TL_FLAG_PDL) != 0;
+    return plan->fmt == TL_FMT_2BIT
+               ? tlk::launch_gemvp<2>(a, dev->num_sms, pdl, (cudaStream_t)stream,
+                                      &t_last_cuda_error)
+               : tlk::launch_gemvp<16>(a, dev->num_sms, pdl, (cudaStream_t)stream,
+                                       &t_last_cuda_error);
 }
 
 int tl_device_status(void *stream) {

@@ -18,6 +18,14 @@
 //    mbarriers that recycle the ring stages;
 //  * the decode warps then read the accumulator with tcgen05.ld, scale by
 //    alpha and store fp16.
+// Split-K, for shapes with fewer output tiles than SMs: a cluster of S CTAs
+// shares one output tile, rank r taking K-steps [r nk / S, (r + 1) nk / S).
+// After one cluster barrier (every ring is then idle), the accumulator is
+// cut into units of 32 rows (a TMEM lane quarter) x 32 columns; unit u is
+// owned by rank u mod S.  Each CTA pushes the units it does not own from
+// TMEM into the owner's activation ring with st.async, and the owner sums
+// the S partials of its units in rank order -- deterministic, no global
+// workspace.
 // Every mbarrier wait is bounded; a timeout sets the device error word.
 #pragma once
 #include <cuda.h>
@@ -77,12 +85,20 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     uint64_t *afull = full + kGemmStages;   // decoders -> MMA (A stage written)
     uint64_t *empty = afull + kGemmStages;  // MMA commit -> producer / decoders
     uint64_t *done = empty + kGemmStages;   // last MMA committed -> epilogue
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(done + 1);
+    uint64_t *redbar = done + 1;            // split-K: the partials pushed to this CTA landed
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(redbar + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kGemmRows;
     const int m0 = blockIdx.y * BN;
-    const int nk = (K + kGemmKStep - 1) / kGemmKStep;
+    const int nk_all = (K + kGemmKStep - 1) / kGemmKStep;
+    // split-K rank and K-step range (the host keeps S <= nk_all, so no range is empty)
+    const uint32_t S = cluster_nctarank(), rank = cluster_ctarank();
+    const int kb = (int)(((int64_t)nk_all * rank) / S);
+    const int nk = (int)(((int64_t)nk_all * (rank + 1)) / S) - kb;
+    // accumulator units: 4 lane quarters x kChunks column chunks of kChunkW
+    constexpr int kChunkW = BN < 32 ? BN : 32;
+    constexpr int kChunks = (BN + 31) / 32;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
@@ -91,6 +107,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             mbar_init(&empty[s], 1);
         }
         mbar_init(done, 1);
+        mbar_init(redbar, 1);
+        // bytes pushed here: (S - 1) sources x the tile's 128 x BN floats / S
+        if (S > 1) mbar_arrive_expect_tx(redbar, (S - 1) * (uint32_t)(kGemmRows * BN * 4) / S);
         fence_mbar_init();
         tma_prefetch_desc(&tmap_w);
         tma_prefetch_desc(&tmap_x);
@@ -114,8 +133,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
                     break;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 tma_load_2d(xs + s * GemmSmem::x_stage_bytes(BN), &tmap_x, &full[s],
-                            k * kGemmKStep, m0);
-                tma_load_2d(ws + s * GemmSmem::w_stage_bytes, &tmap_w, &full[s], k * 16, n0);
+                            (kb + k) * kGemmKStep, m0);
+                tma_load_2d(ws + s * GemmSmem::w_stage_bytes, &tmap_w, &full[s], (kb + k) * 16,
+                            n0);
             }
             // drain: make sure every issued copy has landed before the CTA may exit
             for (int k = nk - kGemmStages > 0 ? nk - kGemmStages : 0; k < nk; ++k) {
@@ -174,8 +194,9 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             mbar_arrive(&afull[s]);
         }
         // ---- epilogue: accumulator -> alpha -> fp16 -> Y ----
-        if (ok) ok = mbar_wait(done, 0);
-        if (ok) {
+        // (split-K waits for the MMAs as well: TMEM and the ring are reused below)
+        const bool fin = mbar_wait(done, 0);
+        if (S == 1 && ok && fin) {
             tc_fence_after();
             const int n = n0 + row;
 #pragma unroll 1
@@ -194,6 +215,84 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             }
         }
     }
+    if (S > 1) {
+        // every CTA of the cluster has finished its MMAs, so its activation ring
+        // is idle and can take the partials; the proxy fence orders the tensor
+        // core's reads of the ring before the stores that will overwrite it
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        cluster_sync();
+        if (warp >= 2) {
+            tc_fence_after();
+            const int quarter = warp & 3;
+            const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+            const int per = 4 * kChunks / (int)S;  // units owned per rank
+            const uint32_t xs_addr = smem_u32(xs);
+            // push: unit u = quarter * kChunks + c goes to rank u % S, slot
+            // [source rank][u / S][kChunkW / 4 groups of 4 floats][32 lanes]
+#pragma unroll 1
+            for (int c = 0; c < kChunks; ++c) {
+                const int u = quarter * kChunks + c;
+                const uint32_t owner = (uint32_t)u % S;
+                if (owner == rank) continue;
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + lane_addr + c * 32, v);
+                tc_wait_ld();
+                const uint32_t slot = rank * per + (uint32_t)u / S;
+                const uint32_t dst = mapa_shared(
+                    xs_addr + (slot * (kChunkW / 4) * 32 + lane) * 16u, owner);
+                const uint32_t rbar = mapa_shared(smem_u32(redbar), owner);
+#pragma unroll
+                for (int c4 = 0; c4 < kChunkW / 4; ++c4)
+                    st_async_v4_f32_mapped(dst + c4 * 32 * 16, rbar, __uint_as_float(v[4 * c4]),
+                                           __uint_as_float(v[4 * c4 + 1]),
+                                           __uint_as_float(v[4 * c4 + 2]),
+                                           __uint_as_float(v[4 * c4 + 3]));
+            }
+            // reduce the units this CTA owns, in rank order
+            if (mbar_wait_cluster(redbar, 0)) {
+                const int n = n0 + quarter * 32 + lane;
+#pragma unroll 1
+                for (int c = 0; c < kChunks; ++c) {
+                    const int u = quarter * kChunks + c;
+                    if ((uint32_t)u % S != rank) continue;
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + lane_addr + c * 32, v);
+                    tc_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < kChunkW / 4; ++c4) {
+                        float a[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (uint32_t r = 0; r < S; ++r) {
+                            float4 p;
+                            if (r == rank) {
+                                p = make_float4(__uint_as_float(v[4 * c4]),
+                                                __uint_as_float(v[4 * c4 + 1]),
+                                                __uint_as_float(v[4 * c4 + 2]),
+                                                __uint_as_float(v[4 * c4 + 3]));
+                            } else {
+                                const uint32_t slot = r * per + (uint32_t)u / S;
+                                p = *reinterpret_cast<const float4 *>(
+                                    xs + (slot * (kChunkW / 4) * 32 + c4 * 32 + lane) * 16u);
+                            }
+                            a[0] += p.x;
+                            a[1] += p.y;
+                            a[2] += p.z;
+                            a[3] += p.w;
+                        }
+                        if (n < N) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int m = m0 + c * 32 + 4 * c4 + j;
+                                if (m < M)
+                                    Y[(int64_t)m * ldy + n] = f32_to_f16_bits(alpha * a[j]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -205,9 +304,65 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 }
 
 // ---- host side ---------------------------------------------------------------
+// Every CTA asks for more than half of an SM's 228 KB of shared memory, so at
+// most one CTA of this kernel (of any BN, from any number of concurrent
+// launches) is resident per SM and its TMEM allocation (<= 512 columns) never
+// waits.  tcgen05.alloc blocks while columns are taken; with split-K clusters
+// such a wait could close a cycle (a CTA holding TMEM at the cluster barrier
+// for a peer that waits for TMEM behind it).
+constexpr size_t kGemmMinSmem = 116 * 1024 + 1;
 inline size_t gemm_smem_bytes(int bn) {
-    return 1024 + kGemmStages * ((size_t)bn * 128 + kGemmRows * 16) + (3 * kGemmStages + 1) * 8 +
-           16;
+    const size_t need = 1024 + kGemmStages * ((size_t)bn * 128 + kGemmRows * 16) +
+                        (3 * kGemmStages + 2) * 8 + 16;
+    return need > kGemmMinSmem ? need : kGemmMinSmem;
+}
+
+// CTAs of gemm2_kernel<BN> that can be resident at once in clusters of S
+// (cached per device and S; -1 if the occupancy query fails).
+template <int BN>
+inline int gemm_resident(int dev, int S, size_t smem) {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static int cache[kMaxDev][4] = {};  // S = 1, 2, 4, 8; 0 = not queried yet
+    const int si = S == 1 ? 0 : S == 2 ? 1 : S == 4 ? 2 : 3;
+    if (dev < 0 || dev >= kMaxDev) return -1;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (cache[dev][si] != 0) return cache[dev][si];
+    }
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(1, 1, 1024);
+    q.blockDim = dim3(kGemmThreads);
+    q.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = (unsigned)S;
+    q.attrs = at;
+    q.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm2_kernel<BN>, &q) != cudaSuccess) return -1;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[dev][si] = clusters * S > 0 ? clusters * S : -1;
+    return cache[dev][si];
+}
+
+// Split-K factor: the largest S in {1, 2, 4, 8} such that the S-CTA clusters
+// of all output tiles are resident at once, S divides the accumulator's
+// 4 x ceil(BN / 32) units and every rank keeps at least one K-step.
+template <int BN>
+inline int gemm_split(int dev, int M, int N, int K, size_t smem) {
+    const int64_t tiles = (int64_t)((N + kGemmRows - 1) / kGemmRows) * ((M + BN - 1) / BN);
+    const int units = 4 * ((BN + 31) / 32);
+    const int nk = (K + kGemmKStep - 1) / kGemmKStep;
+    int S = 1;
+    while (2 * S <= 8 && units % (2 * S) == 0 && 2 * S <= nk) {
+        const int r = gemm_resident<BN>(dev, 2 * S, smem);
+        if (r <= 0 || tiles * 2 * S > r) break;
+        S *= 2;
+    }
+    return S;
 }
 
 template <int BN>
@@ -259,9 +414,22 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
         *last_cuda_error = (int)attr_err[dev];
         return 5;
     }
-    dim3 grid((unsigned)((N + kGemmRows - 1) / kGemmRows), (unsigned)((M + BN - 1) / BN));
-    gemm2_kernel<BN><<<grid, kGemmThreads, smem, stream>>>(tw, tx, alpha, dY, ldy, M, N, K);
-    cudaError_t e = cudaGetLastError();
+    const int S = gemm_split<BN>(dev, M, N, K, smem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((N + kGemmRows - 1) / kGemmRows), (unsigned)((M + BN - 1) / BN),
+                       (unsigned)S);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = (unsigned)S;
+    cfg.attrs = at;
+    cfg.numAttrs = S > 1 ? 1 : 0;  // S = 1: a plain launch
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN>, tw, tx, alpha, dY, ldy, M, N, K);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;
         return 5;

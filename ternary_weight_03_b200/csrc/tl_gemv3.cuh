@@ -298,7 +298,7 @@ gemv3_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restr
         }
     }
     if (S > 1)
-        mbar_wait(redbar, 0);  // all S x (tiles owned) partials have arrived
+        mbar_wait_cluster(redbar, 0);  // all S x (tiles owned) partials have arrived
     else
         __syncthreads();
     {

@@ -67,6 +67,34 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
 }
 
+// The same bounded wait with acquire semantics at cluster scope, for phases
+// completed by other CTAs of the cluster (st.async complete_tx), so their
+// stores into this CTA's shared memory are visible after it returns true.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_error_word, kErrTimeout);
+            return false;
+        }
+    }
+}
+
 // ---- TMA (tensor tile loads, no multicast) ---------------------------------
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar,
                                             int x, int y) {
@@ -210,6 +238,23 @@ __device__ __forceinline__ void st_async_v2_f32(uint32_t local_addr, uint32_t ra
         "st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(
             raddr),
         "f"(a), "f"(b), "r"(rbar)
+        : "memory");
+}
+// Address in CTA `rank`'s shared-memory window of the location that is
+// `local_addr` in this CTA.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+    return r;
+}
+// Four floats to an address already mapped into another CTA's window,
+// completing 16 bytes on the (mapped) mbarrier `remote_bar` there.
+__device__ __forceinline__ void st_async_v4_f32_mapped(uint32_t remote_addr, uint32_t remote_bar,
+                                                       float a, float b, float c, float d) {
+    asm volatile(
+        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, "
+        "[%5];" ::"r"(remote_addr),
+        "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
         : "memory");
 }
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t local_addr, uint32_t rank) {

@@ -84,3 +84,75 @@ def test_gemv_ex_flags(L):
     # unknown flag bits are rejected before anything reaches a device
     assert L.tl_gemv_ex(2, A_, 256, 1.0, A_, 1024, A_, 1024, 1, 1024, 1024, 2, None) == 1
     assert L.tl_gemv_ex(2, A_, 256, 1.0, A_, 1024, A_, 1024, 9, 1024, 1024, 1, None) == 1
+
+
+def _layers(specs):
+    """ctypes layers with fake, aligned device addresses (never dereferenced)."""
+    arr = (tl.Layer * len(specs))()
+    for i, sp in enumerate(specs):
+        d = dict(dT=A, ldp=256, alpha=0.5, dX=A, ldx=1024, dY=A, ldy=1024, M=1, N=1024, K=1024,
+                 flags=0)
+        d.update(sp)
+        arr[i] = tl.Layer(**d)
+    return arr
+
+
+def _ws(L, fmt, arr):
+    import ctypes
+    n = ctypes.c_size_t(0)
+    rc = L.tl_gemv_batch_bytes(fmt, len(arr), arr, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_batch_workspace_size(L):
+    # table (one 88-byte entry + one 128-byte TMA descriptor per layer), counters,
+    # and fp32 partials only for layers whose rows are split across CTAs
+    rc, n = _ws(L, 2, _layers([dict(N=1000, K=2048, ldp=512, ldx=2048, ldy=1000)]))
+    assert rc == 0 and n == 1024  # header 256, table 256, map 256, 9 tile counters 256
+    rc1, n1 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096, M=1)]))
+    rc8, n8 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096, M=8)]))
+    assert rc1 == rc8 == 0
+    tiles = (4096 + 119) // 120
+    assert n1 > 1024 and n8 > n1
+    # documented bound: ~200 B per layer + ~N * M * 4 * (K / 2048) for a split layer
+    assert n1 <= 2048 + 4096 * 1 * 4 * (14336 // 2048 + 1) * 128 // 120
+    rc2, n2 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096,
+                                      dT=A + 4096)] * 2))
+    assert rc2 == 0 and n2 >= 2 * (n1 - 1024)
+
+
+@pytest.mark.parametrize("spec,count,rc", [
+    (dict(M=0), 1, 1), (dict(M=9), 1, 1), (dict(flags=2), 1, 1), (dict(flags=1), 1, 1),
+    (dict(dT=0), 1, 1), (dict(ldp=255), 1, 1), (dict(dX=A + 2), 1, 4), (dict(ldy=1028), 1, 4),
+    (dict(), 0, 1), (dict(), 4097, 1),
+])
+def test_batch_argument_rules(L, spec, count, rc):
+    arr = _layers([spec] * max(count, 1))
+    import ctypes
+    n = ctypes.c_size_t(0)
+    plan = tl.Plan()
+    assert L.tl_gemv_batch_bytes(2, count, arr, ctypes.byref(n)) == rc
+    assert L.tl_gemv_batch_plan(2, count, arr, A, 1 << 20, ctypes.byref(plan)) == rc
+
+
+def test_batch_plan_and_run_rules(L):
+    import ctypes
+    arr = _layers([dict(), dict(flags=1)])  # layer 1 may read layer 0's output
+    rc, n = _ws(L, 2, arr)
+    assert rc == 0
+    plan = tl.Plan()
+    pp = ctypes.byref(plan)
+    assert L.tl_gemv_batch_plan(2, 2, arr, 0, n, pp) == 1          # no workspace
+    assert L.tl_gemv_batch_plan(2, 2, arr, A + 16, n, pp) == 4     # not 256-byte aligned
+    assert L.tl_gemv_batch_plan(2, 2, arr, A, n - 1, pp) == 1      # too small
+    assert L.tl_gemv_batch_plan(3, 2, arr, A, n, pp) == 1          # unknown format
+    assert L.tl_gemv_batch_plan(2, 2, arr, A, n, None) == 1        # no plan
+    # run refuses a plan that tl_gemv_batch_plan did not fill
+    assert L.tl_gemv_batch_run(None, 0, None) == 1
+    assert L.tl_gemv_batch_run(pp, 0, None) == 1
+    bad = tl.Plan(fmt=2, count=2, max_m=9, total_items=3, total_tiles=2, dWorkspace=A,
+                  workspace_bytes=n)
+    assert L.tl_gemv_batch_run(ctypes.byref(bad), 0, None) == 1
+    good = tl.Plan(fmt=2, count=2, max_m=1, total_items=3, total_tiles=2, dWorkspace=A,
+                   workspace_bytes=n)
+    assert L.tl_gemv_batch_run(ctypes.byref(good), 8, None) == 1   # unknown flag

@@ -1,0 +1,261 @@
+"""tl_gemv_batch_plan / tl_gemv_batch_run (one persistent launch over many
+decode-shaped layers) on the GPU against the oracle, layer by layer.
+
+Tolerance per element, as for tl_gemv: |y - y_ref| <= 1e-3 * alpha *
+sum_k |x[m,k]| + ulp16(y_ref).  Chained layers (TL_LAYER_READS_EARLIER) are
+checked against the oracle applied layer by layer on the intermediate as the
+GPU stores it (binary16), the bound adding alpha * sum_k ulp16(x_k) for the
+one-ulp freedom of each stored intermediate.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from ternary_weight_03_b200 import build
+    build.build()
+
+
+def _device_layer(fmt, T, X, ldp_extra=0, ldx_extra=0, ldy_extra=0):
+    """Upload one layer with junk in every padding byte / element (0xFF codes,
+    NaN activations, NaN outputs) and one guard row below Y."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    N, K = T.shape
+    M = X.shape[0]
+    ldp = tl.padded_ldp(fmt, K) + 16 * ldp_extra
+    P = tl.pack(fmt, T, ldp=ldp)
+    P[:, tl.row_bytes(fmt, K):] = 0xFF
+    ldx = K + (-K) % 8 + 8 * ldx_extra
+    Xh = np.full((M, ldx), np.nan, dtype=np.float16)
+    Xh[:, :K] = X
+    ldy = N + (-N) % 8 + 8 * ldy_extra
+    dY = torch.full((M + 1, ldy), float("nan"), dtype=torch.float16, device="cuda")
+    return torch.from_numpy(P).cuda(), torch.from_numpy(Xh).cuda(), dY
+
+
+def _check_layer(T, X, a, dY, N, M):
+    Y = dY.cpu().numpy()
+    assert np.isnan(Y[M, :].astype(np.float32)).all(), "wrote past row M"
+    if Y.shape[1] > N:
+        assert np.isnan(Y[:M, N:].astype(np.float32)).all(), "wrote past column N"
+    got = Y[:M, :N].astype(np.float64)
+    ref = oracle.get().linear(T, X, a, nthreads=8)
+    tol = oracle.tolerance(ref, X, a)
+    err = np.abs(got - ref)
+    assert (err <= tol).all(), f"{int((err > tol).sum())} of {err.size} outside tolerance"
+
+
+def _plan(fmt, layers):
+    """Workspace + plan of a batch (the workspace must outlive the plan)."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    nbytes = tl.gemv_batch_bytes(fmt, layers)
+    ws = torch.full((nbytes,), 0xAB, dtype=torch.uint8, device="cuda")  # junk: plan clears
+    return tl.gemv_batch_plan(fmt, layers, ws), ws
+
+
+def _counters_zero(ws):
+    return not ws[:256].cpu().numpy().any()
+
+
+# (M, N, K, p0): ragged N and K (tails inside a byte, a group and a K-part),
+# single rows and columns, long rows split into many K-parts
+MIXED = [(1, 1, 1, 1 / 3), (3, 7, 5, 0.2), (8, 121, 255, 0.6), (2, 250, 257, 1 / 3),
+         (1, 240, 1000, 1 / 3), (5, 130, 2049, 0.2), (1, 300, 4100, 1 / 3), (8, 64, 14336, 1 / 3),
+         (1, 1000, 3072, 0.6), (4, 129, 8200, 1 / 3)]
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+def test_mixed_independent_layers(fmt):
+    import ternary_weight_03_b200 as tl
+    cases, specs = [], []
+    for i, (M, N, K, p0) in enumerate(MIXED):
+        T = synth.trits(100 + i, N, K, p0=p0)
+        X = synth.activations(200 + i, M, K)
+        a = synth.alpha_for(300 + i)
+        dP, dX, dY = _device_layer(fmt, T, X, ldp_extra=i % 2, ldx_extra=i % 3, ldy_extra=i % 2)
+        cases.append((T, X, a, dP, dX, dY))
+        specs.append((dP, a, dX, K, dY))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    outs = []
+    for rep in range(3):  # the plan is run again without clearing anything
+        for c in cases:
+            c[5].fill_(float("nan"))
+        tl.gemv_batch_run(plan)
+        assert tl.device_status() == 0
+        outs.append([c[5].cpu().numpy().view(np.uint16).copy() for c in cases])
+        assert _counters_zero(ws), "workspace counters not reset"
+    for r in outs[1:]:
+        for a_, b_ in zip(outs[0], r):
+            assert np.array_equal(a_, b_), "not deterministic"
+    for (T, X, a, dP, dX, dY), (M, N, K, _) in zip(cases, MIXED):
+        _check_layer(T, X, a, dY, N, M)
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+@pytest.mark.parametrize("graph", [False, True])
+def test_chain_reads_earlier(fmt, graph):
+    """Layer i + 1 reads layer i's output (TL_LAYER_READS_EARLIER), under PDL."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    M = 3
+    dims = [3072, 1000, 4096, 257, 2048]  # K of layer 0, then each layer's N
+    Ts = [synth.trits(40 + i, dims[i + 1], dims[i]) for i in range(len(dims) - 1)]
+    X0 = synth.activations(50, M, dims[0])
+    alphas = [0.02, 0.03, 0.015, 0.05]
+    import ternary_weight_03_b200 as tl
+    dX0 = torch.from_numpy(X0).cuda()
+    ys = [torch.full((M, d + (-d) % 8), float("nan"), dtype=torch.float16, device="cuda")
+          for d in dims[1:]]
+    specs = []
+    for i, T in enumerate(Ts):
+        dP = torch.from_numpy(tl.pack(fmt, T)).cuda()
+        X = dX0 if i == 0 else ys[i - 1]
+        specs.append((dP, alphas[i], X, dims[i], ys[i], 0 if i == 0 else tl.LAYER_READS_EARLIER))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        tl.gemv_batch_run(plan, stream=s, flags=tl.FLAG_PDL)
+        torch.cuda.synchronize()
+        if graph:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                tl.gemv_batch_run(plan, stream=s, flags=tl.FLAG_PDL)
+                tl.gemv_batch_run(plan, stream=s, flags=tl.FLAG_PDL)
+            for y in ys:
+                y.fill_(float("nan"))
+            torch.cuda.synchronize()
+            g.replay()
+        else:
+            for y in ys:
+                y.fill_(float("nan"))
+            torch.cuda.synchronize()
+            for _ in range(2):
+                tl.gemv_batch_run(plan, stream=s, flags=tl.FLAG_PDL)
+    torch.cuda.synchronize()
+    assert tl.device_status(s) == 0
+    o = oracle.get()
+    x = X0
+    for i, T in enumerate(Ts):
+        N = dims[i + 1]
+        got = ys[i][:, :N].float().cpu().numpy().astype(np.float64)
+        ref = o.linear(T, x, alphas[i], nthreads=8)
+        tol = oracle.tolerance(ref, x, alphas[i])
+        if i > 0:
+            ulp = np.spacing(np.abs(x).astype(np.float16)).astype(np.float64)
+            tol = tol + abs(alphas[i]) * ulp.sum(axis=1)[:, None]
+        assert (np.abs(got - ref) <= tol).all(), f"layer {i}"
+        x = ys[i][:, :N].cpu().numpy()  # the stored intermediate feeds the next reference
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+def test_sweep_batch_sampled(fmt):
+    """The decode sweep's six matrices at M = 1 and 8 as one 12-layer batch;
+    sampled outputs per layer against the oracle computed one by one."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    sweep = [(3072, 3072), (3072, 8192), (8192, 3072), (4096, 4096), (4096, 14336),
+             (14336, 4096)]
+    specs, cases = [], []
+    for M in (1, 8):
+        for i, (K, N) in enumerate(sweep):
+            T = synth.trits(i, N, K)
+            X = synth.activations(10 * M + i, M, K)
+            a = synth.alpha_for(i)
+            dP = torch.from_numpy(tl.pack(fmt, T)).cuda()
+            dX = torch.from_numpy(X).cuda()
+            dY = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+            specs.append((dP, a, dX, K, dY))
+            cases.append((T, X, a, dY))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+    assert tl.device_status() == 0
+    rng = np.random.default_rng(fmt)
+    o = oracle.get()
+    for T, X, a, dY in cases:
+        Y = dY.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(Y).all()
+        M, N = Y.shape
+        ms = np.concatenate([rng.integers(0, M, 400), [0, M - 1]])
+        ns = np.concatenate([rng.integers(0, N, 400), [0, N - 1]])
+        ref = o.linear_at(T, X, a, ms, ns)
+        tol = oracle.tolerance(ref, X[ms], a)
+        assert (np.abs(Y[ms, ns] - ref) <= tol).all()
+
+
+def test_batch_matches_single_calls():
+    """Every layer of a batch equals tl_gemv's result within the tolerance of
+    both, and the batch is bit-identical across calls."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    specs, singles, cases = [], [], []
+    for i, (M, N, K) in enumerate([(1, 512, 4096), (8, 360, 1536), (2, 1000, 700)]):
+        T = synth.trits(60 + i, N, K)
+        X = synth.activations(70 + i, M, K)
+        dP = torch.from_numpy(tl.pack(2, T)).cuda()
+        Xp = np.zeros((M, K + (-K) % 8), np.float16)  # row stride a multiple of 8
+        Xp[:, :K] = X
+        dX = torch.from_numpy(Xp).cuda()
+        dY = torch.empty((M, N + (-N) % 8), dtype=torch.float16, device="cuda")
+        specs.append((dP, 0.02, dX, K, dY))
+        singles.append(tl.gemv(2, dP, 0.02, dX, K).clone())
+        cases.append((T, X))
+    layers = tl.make_layers(2, specs)
+    plan, ws = _plan(2, layers)
+    tl.gemv_batch_run(plan)
+    torch.cuda.synchronize()
+    for (dP, a, dX, K, dY), ys, (T, X) in zip(specs, singles, cases):
+        N = dP.shape[0]
+        got = dY[:, :N].float().cpu().numpy().astype(np.float64)
+        ref = oracle.get().linear(T, X, a, nthreads=8)
+        tol = oracle.tolerance(ref, X, a)
+        assert (np.abs(got - ref) <= tol).all()
+        assert (np.abs(got - ys.float().cpu().numpy()) <= 2 * tol).all()
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+def test_long_chain_multiple_items_per_cta(fmt):
+    """Eight chained 4096 x 4096 layers: 280 items, more than one per CTA, so a
+    CTA holds stages of layer l while its next item waits for layer l."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    M, D, depth = 2, 4096, 8
+    Ts = [synth.trits(80 + i, D, D) for i in range(depth)]
+    X0 = synth.activations(90, M, D)
+    alphas = [0.02] * depth
+    dX0 = torch.from_numpy(X0).cuda()
+    ys = [torch.full((M, D), float("nan"), dtype=torch.float16, device="cuda")
+          for _ in range(depth)]
+    specs = []
+    for i, T in enumerate(Ts):
+        dP = torch.from_numpy(tl.pack(fmt, T)).cuda()
+        specs.append((dP, alphas[i], dX0 if i == 0 else ys[i - 1], D, ys[i],
+                      0 if i == 0 else tl.LAYER_READS_EARLIER))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+    assert tl.device_status() == 0
+    o = oracle.get()
+    x = X0
+    for i, T in enumerate(Ts):
+        got = ys[i].float().cpu().numpy().astype(np.float64)
+        ref = o.linear(T, x, alphas[i], nthreads=8)
+        tol = oracle.tolerance(ref, x, alphas[i])
+        if i > 0:
+            ulp = np.spacing(np.abs(x).astype(np.float16)).astype(np.float64)
+            tol = tol + abs(alphas[i]) * ulp.sum(axis=1)[:, None]
+        assert (np.abs(got - ref) <= tol).all(), f"layer {i}"
+        x = ys[i].cpu().numpy()

@@ -35,6 +35,20 @@ def test_small_ragged(M, N, K):
     check_against_oracle(T, X, a, Y)
 
 
+# Few output tiles: the kernel splits K over a cluster of 2 to 8 CTAs (one
+# K-step per rank at K = 256 / 200, uneven ranges at K = 520) and reduces the
+# partials in rank order, so repeated calls must agree bit for bit.
+SPLIT_K = [(64, 1000, 2048), (256, 512, 256), (16, 640, 1000), (32, 300, 200),
+           (128, 2048, 520), (512, 1024, 4096), (96, 129, 777)]
+
+
+@pytest.mark.parametrize("M,N,K", SPLIT_K)
+def test_split_k(M, N, K):
+    T, X, a = make_case(2, M, N, K, seed=M + 3 * N + 7 * K)
+    Y, _ = run_layer(2, T, X, a, fn="tl_gemm", repeat=3)
+    check_against_oracle(T, X, a, Y)
+
+
 @pytest.mark.parametrize("extra", [(1, 0, 0), (0, 2, 0), (0, 0, 3)])
 def test_strides(extra):
     T, X, a = make_case(2, 40, 200, 300, seed=5)
@@ -78,7 +92,7 @@ def _sampled(M, N, K, seed, samples=3000):
 
 
 @pytest.mark.parametrize("M", [16, 64, 256, 1024, 4096])
-@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
+@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096), (4096, 4096)])
 def test_prefill_shapes_sampled(M, K, N):
     _sampled(M, N, K, seed=M + K)
 
