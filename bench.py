@@ -190,6 +190,30 @@ class Sweep:
         self.bytes_per_step = self.bytes_per_pass * len(ms)
         self.launches_per_step = len(self.items) * len(ms)
         self.rotation_bytes = self.copies * per_set
+        self.batch = False
+        self.plans, self.workspaces = [], []
+
+    def use_batch(self):
+        """Switch to one tl_gemv_batch_run per step: every layer of the step in a
+        single launch.  Phase ph's plan reads the M-th token count's weights from
+        copy (len(ms) * ph + m) % copies, the same rotation as the per-call steps."""
+        import torch
+        import ternary_weight_03_b200 as tl
+        nm = len(self.ms)
+        nphase = self.copies // nm if self.copies % nm == 0 else self.copies
+        for ph in range(nphase):
+            specs = []
+            for mi, M in enumerate(self.ms):
+                copy = (nm * ph + mi) % self.copies
+                for i, (K, N, _, alpha, xs) in enumerate(self.items):
+                    specs.append((self.dP[copy][i], alpha, xs[M], K, self.Y[M][i]))
+            layers = tl.make_layers(self.fmt, specs)
+            ws = torch.zeros(tl.gemv_batch_bytes(self.fmt, layers), dtype=torch.uint8,
+                             device=self.dev)
+            self.plans.append(tl.gemv_batch_plan(self.fmt, layers, ws))
+            self.workspaces.append(ws)
+        self.batch = True
+        self.launches_per_step = 1
 
     def enqueue(self, step: int, stream, events=None, flags: int = 1):
         """Enqueue the calls of one step on `stream` (optionally recording an
@@ -197,6 +221,13 @@ class Sweep:
         each call may start streaming its (static) weights while the previous
         call drains."""
         import ternary_weight_03_b200 as tl
+        if self.batch:
+            if events is not None:
+                events[0].record(stream)
+            tl.gemv_batch_run(self.plans[step % len(self.plans)], stream=stream, flags=flags)
+            if events is not None:
+                events[1].record(stream)
+            return
         L = tl.lib()
         s = stream.cuda_stream
         j = 0
@@ -226,6 +257,8 @@ def time_graphs(sweep: Sweep, steps: int, warmup: int, stream, clock_gpu: int | 
     import torch
     nm = len(sweep.ms)
     nphase = sweep.copies // nm if sweep.copies % nm == 0 else sweep.copies
+    if sweep.batch:
+        nphase = len(sweep.plans)
     graphs = []
     with torch.cuda.stream(stream):
         sweep.enqueue(0, stream, flags=flags)  # per-device setup outside capture
@@ -273,32 +306,35 @@ def time_graphs(sweep: Sweep, steps: int, warmup: int, stream, clock_gpu: int | 
 
 def time_e2e(sweep: Sweep, steps: int, warmup: int, stream):
     """End to end through the C ABI from pinned host buffers: every step
-    copies its packed weights and activations host -> device, runs the twelve
-    calls and copies the outputs back.  Returns (ms, h2d bytes, d2h bytes)."""
+    copies its packed weights and activations host -> device, runs the step's
+    layers in one tl_gemv_batch_run (planned once on these buffers) and copies
+    the outputs back.  Returns (ms, h2d bytes, d2h bytes)."""
     import torch
     import ternary_weight_03_b200 as tl
-    L = tl.lib()
     hP = [torch.from_numpy(P).pin_memory() for (_, _, P, _, _) in sweep.items]
     hX = {M: [xs[M].cpu().pin_memory() for (_, _, _, _, xs) in sweep.items] for M in sweep.ms}
     hY = {M: [torch.empty(tuple(y.shape), dtype=torch.float16).pin_memory() for y in sweep.Y[M]]
           for M in sweep.ms}
-    dP = [torch.empty_like(p, device=sweep.dev) for p in hP]
+    # one device copy of the weights per token count, as in the device-resident step
+    dP = {M: [torch.empty_like(p, device=sweep.dev) for p in hP] for M in sweep.ms}
     dX = {M: [torch.empty_like(x, device=sweep.dev) for x in hX[M]] for M in sweep.ms}
+    specs = [(dP[M][i], alpha, dX[M][i], K, sweep.Y[M][i])
+             for M in sweep.ms for i, (K, N, _, alpha, _) in enumerate(sweep.items)]
+    layers = tl.make_layers(sweep.fmt, specs)
+    ws = torch.zeros(tl.gemv_batch_bytes(sweep.fmt, layers), dtype=torch.uint8, device=sweep.dev)
+    plan = tl.gemv_batch_plan(sweep.fmt, layers, ws)
     h2d = sum(p.numel() for p in hP) * len(sweep.ms) + sum(
         x.numel() * 2 for M in sweep.ms for x in hX[M])
     d2h = sum(y.numel() * 2 for M in sweep.ms for y in hY[M])
 
     def one_step():
         for M in sweep.ms:
-            for i, (K, N, _, alpha, _) in enumerate(sweep.items):
-                dP[i].copy_(hP[i], non_blocking=True)
+            for i in range(len(sweep.items)):
+                dP[M][i].copy_(hP[i], non_blocking=True)
                 dX[M][i].copy_(hX[M][i], non_blocking=True)
-                Y = sweep.Y[M][i]
-                rc = L.tl_gemv(sweep.fmt, dP[i].data_ptr(), dP[i].stride(0), alpha,
-                               dX[M][i].data_ptr(), dX[M][i].stride(0), Y.data_ptr(), Y.stride(0),
-                               M, N, K, stream.cuda_stream)
-                if rc != 0:
-                    raise RuntimeError(f"tl_gemv -> {tl.status_str(rc)}")
+        tl.gemv_batch_run(plan, stream=stream)
+        for M in sweep.ms:
+            for i, Y in enumerate(sweep.Y[M]):
                 hY[M][i].copy_(Y, non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -379,59 +415,63 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     """All linear layers of one decode step of a 30-layer LLaMA-style SwiGLU
     decoder (hidden 3072, intermediate 8192): per layer q, k, v, o
     (3072 -> 3072), gate, up (3072 -> 8192), down (8192 -> 3072), i.e. 210
-    distinct seeded matrices (p0 = 1/3, alpha ~ U(0.01, 0.05)) run back to back
-    in one CUDA graph with programmatic dependent launch.  Each layer gets its
-    own seeded activation vector(s).  Returns GB/s of packed weights."""
+    distinct seeded matrices (p0 = 1/3, alpha ~ U(0.01, 0.05)), each with its
+    own seeded activation vector(s), run as ONE tl_gemv_batch_run per step
+    (graph-captured, programmatic dependent launch).  "chained" reruns the
+    2-bit M = 1 step with every layer flagged as reading the earlier layers'
+    outputs (a serial dependency per layer).  Returns GB/s of packed weights."""
     import torch
     import synth
     import ternary_weight_03_b200 as tl
-    L = tl.lib()
     mats = []  # (K, N, seed)
     for layer in range(30):
         for j, (_, K, N) in enumerate(DECODE_LAYER):
             mats.append((K, N, 1000 + 7 * layer + j))
     out = {}
+
+    def timed(plan):
+        with torch.cuda.stream(stream):
+            tl.gemv_batch_run(plan, stream=stream, flags=1)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                tl.gemv_batch_run(plan, stream=stream, flags=1)
+            for _ in range(warmup):
+                g.replay()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            a.record(stream)
+            for _ in range(steps):
+                g.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
     for fmt in fmts:
         dev_mats, total = [], 0
         for (K, N, seed) in mats:
-            T = synth.trits(seed, N, K)
-            P = tl.pack(fmt, T)
+            P = tl.pack(fmt, synth.trits(seed, N, K))
             dev_mats.append((K, N, torch.from_numpy(P).to(dev), synth.alpha_for(seed)))
             total += N * tl.row_bytes(fmt, K)
         for M in ms:
             xs = [torch.from_numpy(synth.activations(seed, M, K)).to(dev)
                   for (K, N, seed) in mats]
             ys = [torch.empty((M, N), dtype=torch.float16, device=dev) for (K, N, _) in mats]
-
-            def enqueue():
-                for (K, N, dP, alpha), X, Y in zip(dev_mats, xs, ys):
-                    rc = L.tl_gemv_ex(fmt, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(),
-                                      X.stride(0), Y.data_ptr(), Y.stride(0), M, N, K, 1,
-                                      stream.cuda_stream)
-                    if rc != 0:
-                        raise RuntimeError(tl.status_str(rc))
-
-            with torch.cuda.stream(stream):
-                enqueue()
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    enqueue()
-                for _ in range(warmup):
-                    g.replay()
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                torch.cuda.synchronize()
-                a.record(stream)
-                for _ in range(steps):
-                    g.replay()
-                b.record(stream)
-                torch.cuda.synchronize()
-            ms_step = a.elapsed_time(b) / steps
-            gbs = total / (ms_step * 1e-3) / 1e9
-            out[f"fmt{fmt}_M{M}"] = {"packed_bytes": total, "us_per_step": round(ms_step * 1e3, 2),
-                                     "GB/s": round(gbs, 1),
-                                     "frac_hbm": round(gbs / peaks()["hbm_gbs"], 4)}
-            del g, xs, ys
+            variants = [("", 0)] + ([("_chained", tl.LAYER_READS_EARLIER)]
+                                    if fmt == 2 and M == 1 else [])
+            for suffix, flag in variants:
+                specs = [(dP, alpha, X, K, Y, flag if i else 0)
+                         for i, ((K, N, dP, alpha), X, Y) in enumerate(zip(dev_mats, xs, ys))]
+                layers = tl.make_layers(fmt, specs)
+                ws = torch.zeros(tl.gemv_batch_bytes(fmt, layers), dtype=torch.uint8, device=dev)
+                plan = tl.gemv_batch_plan(fmt, layers, ws)
+                ms_step = timed(plan)
+                gbs = total / (ms_step * 1e-3) / 1e9
+                out[f"fmt{fmt}_M{M}{suffix}"] = {
+                    "packed_bytes": total, "us_per_step": round(ms_step * 1e3, 2),
+                    "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks()["hbm_gbs"], 4)}
+                del plan, ws
+            del xs, ys
         del dev_mats
         torch.cuda.empty_cache()
     return out
@@ -443,8 +483,9 @@ def secondary(dev, stream, quick: bool):
     import ternary_weight_03_b200 as tl
     out = {}
     pk = peaks()
-    # 1.6-bit sweep
+    # 1.6-bit sweep, one launch per step
     sw = Sweep(16, dev)
+    sw.use_batch()
     ms, per_launch, _ = time_graphs(sw, 5, 3, stream)
     gbs = sw.bytes_per_step * 5 / (ms * 1e-3) / 1e9
     out["gemv_1p6bit_sweep"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
@@ -483,11 +524,13 @@ def secondary(dev, stream, quick: bool):
                                        "frac_tensor": round(tf / pk["bf16_tflops"], 4)}
     out["gemm_2bit"] = gemm
     out["decode_step_30_layers"] = decode_step(dev, stream)
+    # the same 2-bit sweep as twelve tl_gemv_ex calls per step (with and without PDL)
     sw = Sweep(2, dev)
-    ms, _, _ = time_graphs(sw, 20, 3, stream, flags=0)
-    gbs = sw.bytes_per_step * 20 / (ms * 1e-3) / 1e9
-    out["gemv_2bit_sweep_without_pdl"] = {"GB/s": round(gbs, 1),
-                                          "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
+    for flags, key in ((1, "gemv_2bit_sweep_per_call_pdl"), (0, "gemv_2bit_sweep_per_call")):
+        ms, _, _ = time_graphs(sw, 20, 3, stream, flags=flags)
+        gbs = sw.bytes_per_step * 20 / (ms * 1e-3) / 1e9
+        out[key] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                    "us_per_step": round(ms / 20 * 1e3, 2)}
     return out
 
 
@@ -509,6 +552,7 @@ def run_gpu(args):
     pk = peaks()
 
     sweep = Sweep(2, dev)
+    sweep.use_batch()
     total_ms, per_call, clocks = time_graphs(sweep, args.steps, args.warmup, stream,
                                              clock_gpu=local_rank)
     worst = check_outputs(sweep)
@@ -538,17 +582,18 @@ def run_gpu(args):
         "config": {
             "workload": WORKLOAD,
             "packed_bytes_per_step": sweep.bytes_per_step,
-            "calls_per_step": sweep.launches_per_step,
+            "layers_per_step": len(sweep.items) * len(sweep.ms),
+            "launches_per_step": sweep.launches_per_step,
             "l2": f"inputs larger than L2: {sweep.copies} rotating copies of the packed "
                   f"matrices ({sweep.rotation_bytes / 2**20:.0f} MiB) so every call reads HBM",
             "timing": "CUDA graph per step, CUDA events on the launch stream",
-            "launch": "tl_gemv_ex with TL_FLAG_PDL (programmatic dependent launch; "
-                      "static weights are streamed while the previous call drains)",
+            "launch": "one tl_gemv_batch_run per step (all 12 independent layers in one "
+                      "persistent launch) with TL_FLAG_PDL",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "tlk::gemv3_kernel<2>",
+            "kernel": "tlk::gemvp_kernel<2>",
             "achieved": round(achieved, 2),
             "peak": pk["hbm_gbs"],
             "unit": "GB/s",
@@ -556,7 +601,7 @@ def run_gpu(args):
             "traffic": traffic,
             "algorithmic_bytes_per_launch": sweep.bytes_per_step // sweep.launches_per_step,
             "avg_launch_us": round(avg_launch_ms * 1e3, 3),
-            "per_call_us_without_pdl": [round(t * 1e3, 2) for t in per_call],
+            "launch_us_without_pdl": [round(t * 1e3, 2) for t in per_call],
             "peak_source": f"MEASURED_PEAKS.json hbm_gbs ({pk['source']})",
         },
         "e2e": {"value": round(e2e_bytes / (e2e_max * 1e-3) / 1e9, 3), "unit": "GB/s",
@@ -580,7 +625,7 @@ def run_gpu(args):
 def traffic_per_launch():
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel sources (else None)."""
-    p = ROOT / "profiles" / "gemv2_sweep_traffic.json"
+    p = ROOT / "profiles" / "gemvp2_sweep_traffic.json"
     if not p.exists():
         return None
     try:
@@ -673,6 +718,30 @@ def run_single(fmt: int, K: int, N: int, M: int, reps: int = 4):
     print(json.dumps({"single": [fmt, K, N, M], "checksum": float(Y.float().abs().sum())}))
 
 
+def run_batch_once(fmt: int, M: int, reps: int = 3):
+    """The six sweep shapes at M tokens planned as one batch and run `reps`
+    times through tl_gemv_batch_run, nothing else on the device (for ncu)."""
+    import torch
+    import synth
+    import ternary_weight_03_b200 as tl
+    from ternary_weight_03_b200 import build
+    build.build()
+    specs = []
+    for i, (K, N) in enumerate(SWEEP):
+        P, _, alpha = make_matrix(fmt, K, N, i)
+        specs.append((torch.from_numpy(P).cuda(), alpha,
+                      torch.from_numpy(synth.activations(i, M, K)).cuda(), K,
+                      torch.empty((M, N), dtype=torch.float16, device="cuda")))
+    layers = tl.make_layers(fmt, specs)
+    ws = torch.zeros(tl.gemv_batch_bytes(fmt, layers), dtype=torch.uint8, device="cuda")
+    plan = tl.gemv_batch_plan(fmt, layers, ws)
+    for _ in range(reps):
+        tl.gemv_batch_run(plan)
+    torch.cuda.synchronize()
+    print(json.dumps({"batch_once": [fmt, M], "status": tl.device_status(),
+                      "checksum": float(sum(sp[4].float().abs().sum() for sp in specs))}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -682,9 +751,15 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--batch-once", metavar="FMT,M",
+                    help="plan the six sweep shapes at M tokens as one batch and run it 3 times "
+                         "(a small case for profiling the batch kernel)")
     ap.add_argument("--single", metavar="FMT,K,N,M",
                     help="run one seeded layer call 4 times and exit (for ncu captures)")
     args = ap.parse_args(argv)
+    if args.batch_once:
+        run_batch_once(*[int(v) for v in args.batch_once.split(",")])
+        return
     if args.single:
         run_single(*[int(v) for v in args.single.split(",")])
         return

@@ -271,6 +271,9 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         // Items b, b + G, b + 2G, ... (G CTAs): the next item is known at once, so
         // its layer record is loaded while the current item streams.
         uint32_t stage = 0;
+        int ps = 0;               // ring slot of the next stage
+        uint32_t pph = 0;         // its round's parity
+        bool wrapped = false;     // the ring has been filled once
         int qi = 0;
         bool waited = false, ok = true;
         uint32_t final_seen = 0;  // lower bound of the final-tile counter
@@ -383,17 +386,23 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 __syncwarp();
                 stage += pre;
                 g += kGpSG * pre;
+                ps = pre;
+                if (ps == NS) { ps = 0; pph = 1; wrapped = true; }
                 if (!deps) { ok = false; break; }
             } else if (!wait_deps()) {
                 ok = false;
                 break;
             }
             for (; g < it.g1; g += kGpSG, ++stage) {
-                const int s = (int)(stage % NS);
-                if (stage >= (uint32_t)NS &&
-                    !warp_wait(&empty[s], (uint32_t)((stage / NS) - 1) & 1u)) {
+                const int s = ps;
+                if (wrapped && !warp_wait(&empty[s], pph ^ 1u)) {
                     ok = false;
                     break;
+                }
+                if (++ps == NS) {
+                    ps = 0;
+                    pph ^= 1u;
+                    wrapped = true;
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&wfull[s], kGpWBytes + (uint32_t)L.M * xbytes(g));
@@ -413,17 +422,22 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             mbar_wait(&wfull[t % NS], (t / NS) & 1u);
     } else if (warp == 1) {
         // ---------------- stager ----------------
-        uint32_t stage = 0;
+        int ss = 0;
+        uint32_t sph = 0;
         int qi = 0;
         bool ok = true;
         GpQEntry e;
         while (ok && gp_next_item(queue, qfull, qempty, qi, e)) {
             const int M = e.M, K = e.K;
-            for (int g = e.g0; g < e.g1; g += kGpSG, ++stage) {
-                const int s = (int)(stage % NS);
-                if (!warp_wait(&wfull[s], (uint32_t)(stage / NS) & 1u)) {
+            for (int g = e.g0; g < e.g1; g += kGpSG) {
+                const int s = ss;
+                if (!warp_wait(&wfull[s], sph)) {
                     ok = false;
                     break;
+                }
+                if (++ss == NS) {
+                    ss = 0;
+                    sph ^= 1u;
                 }
                 // activations of this stage below K (and below the item's last group)
                 const int valid = min(K - g * TRITS_GROUP, (e.g1 - g) * TRITS_GROUP);
@@ -553,7 +567,8 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         const int g = lane >> 2, c = lane & 3;
         const bool onesB = (g == 7);
         const int rowA = rt * kG3TileRows + g, rowB = rowA + 8;
-        uint32_t stage = 0;
+        int cs = 0;
+        uint32_t cph = 0;
         int qi = 0, pi = 0;
         bool ok = true;
         GpQEntry e;
@@ -562,12 +577,15 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             float acc[4][4], acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-            for (int gg = e.g0; gg < e.g1; gg += kGpSG, ++stage) {
-                const int s = (int)(stage % NS);
-                const uint32_t par = (uint32_t)(stage / NS) & 1u;
-                if (!warp_wait(&wfull[s], par) || !warp_wait(&xfull[s], par)) {
+            for (int gg = e.g0; gg < e.g1; gg += kGpSG) {
+                const int s = cs;
+                if (!warp_wait(&wfull[s], cph) || !warp_wait(&xfull[s], cph)) {
                     ok = false;
                     break;
+                }
+                if (++cs == NS) {
+                    cs = 0;
+                    cph ^= 1u;
                 }
                 if (gg + h < e.g1) {  // this warp's group exists in the item
                     const uint8_t *box = wring + s * kGpWBytes + h * kGemvGroupBytes + 16 * c;
