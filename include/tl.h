@@ -184,6 +184,28 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
 int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dWorkspace,
                        size_t workspace_bytes, tl_gemv_plan *plan);
 
+/* Bytes of the library's own per-device workspace (see
+ * tl_gemv_batch_plan_static). */
+#define TL_STATIC_WORKSPACE_BYTES (16u << 20)
+
+/* tl_gemv_batch_plan without caller memory: the workspace is a fixed array of
+ * TL_STATIC_WORKSPACE_BYTES bytes inside the library's device code, one per
+ * device, located with cudaGetSymbolAddress on the current device.  Nothing
+ * is allocated.  A batch whose tl_gemv_batch_bytes exceeds
+ * TL_STATIC_WORKSPACE_BYTES is rejected with TL_ERR_INVALID_ARG before
+ * anything is written.  Races: the array is shared by every caller in the
+ * process on that device, so planning again replaces the previous static
+ * plan (a plan filled earlier then runs on the new table); keep one static
+ * plan per device in use at a time and do not plan from several host
+ * threads at once.  The call synchronizes the device first, so no run of an
+ * earlier static plan is still reading the array when it is rewritten.
+ * Clearing: the call zeroes the array's counters; every completed
+ * tl_gemv_batch_run leaves them zero; after a run that ends in
+ * TL_ERR_TIMEOUT, plan again before the next run.  Otherwise as
+ * tl_gemv_batch_plan (blocking, not capturable). */
+int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
+                              tl_gemv_plan *plan);
+
 /* Runs a planned batch in ONE persistent launch: every layer computes
  * exactly what tl_gemv computes.  The launch streams the packed weights of
  * all layers back to back ("What carries the argument": decoding is bound by

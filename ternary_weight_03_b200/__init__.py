@@ -63,6 +63,7 @@ SIGNATURES = {
     "tl_gemv_batch_plan": (_i32, [_i32, _i32, ctypes.POINTER(Layer), _p, ctypes.c_size_t,
                                   ctypes.POINTER(Plan)]),
     "tl_gemv_batch_run": (_i32, [ctypes.POINTER(Plan), ctypes.c_uint, _p]),
+    "tl_gemv_batch_plan_static": (_i32, [_i32, _i32, ctypes.POINTER(Layer), ctypes.POINTER(Plan)]),
     "tl_device_status": (_i32, [_p]),
 }
 
@@ -235,6 +236,18 @@ def gemv_batch_plan(fmt: int, layers, workspace) -> Plan:
            lib().tl_gemv_batch_plan(fmt, len(layers), layers, workspace.data_ptr(),
                                     workspace.numel() * workspace.element_size(),
                                     ctypes.byref(plan)))
+    return plan
+
+
+STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def gemv_batch_plan_static(fmt: int, layers) -> Plan:
+    """Plan a batch into the library's own per-device workspace (no caller
+    memory, nothing allocated; one such plan per device at a time)."""
+    plan = Plan()
+    _check("tl_gemv_batch_plan_static",
+           lib().tl_gemv_batch_plan_static(fmt, len(layers), layers, ctypes.byref(plan)))
     return plan
 
 

@@ -17,6 +17,10 @@ namespace {
 
 thread_local int t_last_cuda_error = 0;
 
+// Workspace of tl_gemv_batch_plan_static: one fixed array per device, part of
+// the library's device image (no allocation call ever creates it).
+__device__ __align__(256) uint8_t g_static_workspace[TL_STATIC_WORKSPACE_BYTES];
+
 int cuda_fail(cudaError_t e) {
     t_last_cuda_error = (int)e;
     return TL_ERR_CUDA;
@@ -212,6 +216,22 @@ int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dW
     plan->dWorkspace = dWorkspace;
     plan->workspace_bytes = workspace_bytes;
     return TL_OK;
+}
+
+int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
+                              tl_gemv_plan *plan) {
+    if (!plan) return TL_ERR_INVALID_ARG;
+    size_t need = 0;
+    int rc = tl_gemv_batch_bytes(fmt, count, layers, &need);
+    if (rc != TL_OK) return rc;
+    if (need > (size_t)TL_STATIC_WORKSPACE_BYTES) return TL_ERR_INVALID_ARG;
+    void *addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_static_workspace);  // this device's copy
+    if (e != cudaSuccess) return cuda_fail(e);
+    // no run of an earlier static plan may still be reading the array
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    return tl_gemv_batch_plan(fmt, count, layers, addr, (size_t)TL_STATIC_WORKSPACE_BYTES, plan);
 }
 
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream) {
