@@ -23,7 +23,7 @@
 // ~40 GB/s per SM that HBM speed needs.)  The per-layer tensor maps and the
 // layer table live in the workspace, written once by tl_gemv_batch_plan.
 //
-// Warp roles of a CTA (608 threads):
+// Warp roles of a CTA (640 threads):
 //  * warp 0, producer: one elected lane issues each stage's copies into a ring
 //    of stages (completion counted in bytes on the stage's mbarrier), claims
 //    items and queues them for the other roles;
@@ -31,11 +31,11 @@
 //    the consumers' layout (2-bit: the pair order of the class-masked decode,
 //    see g3_word2; 1.6-bit: the interleaved units of gemv16_word), with zeros
 //    at k >= K;
-//  * warps 3..18, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
+//  * warps 4..19, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
 //    rows and the all-ones row per warp; warps w and w + 8 take the two K-groups
 //    of each stage for the same rows), accumulating over the item's stages,
 //    then handing the item's 2 x 120 x M sums to
-//  * warp 2, epilogue: y = alpha * (sum - ones-row sum) to Y when the layer has
+//  * warps 2 and 3, epilogues (alternate items): y = alpha * (sum - ones-row sum) to Y when the layer has
 //    one part; otherwise the part's fp32 partial goes to the workspace and the
 //    last of the tile's parts to arrive (per-tile counter) adds the parts in
 //    part order (deterministic) and stores Y.  The tree reduction of per-warp
@@ -56,13 +56,17 @@
 namespace tlk {
 
 constexpr int kGpRowTiles = 8;                               // 15-row tiles per item
-constexpr int kGpSG = 2;                                      // K-groups per stage
-constexpr int kGpConsumers = kGpRowTiles * kGpSG;             // one warp per (tile, group)
-constexpr int kGpWarps = 3 + kGpConsumers;                   // producer, stager, epilogue
-constexpr int kGpThreads = 32 * kGpWarps;                    // 608
+constexpr int kGpConsumers = 2 * kGpRowTiles;                 // two warps per row tile
+constexpr int kGpEpilogues = 2;                               // epilogue warps (alternate items)
+constexpr int kGpWarps = 2 + kGpEpilogues + kGpConsumers;    // + producer, stager
+constexpr int kGpThreads = 32 * kGpWarps;                    // 640
 constexpr int kGpRows = kGpRowTiles * kG3TileRows;            // 120 weight rows per item
-constexpr int kGpStageW = kGpSG * kGemvGroupBytes;            // 128 B per row per stage
-constexpr int kGpWBytes = kGpRows * kGpStageW;                // 15360 B of weights per stage
+// K-groups per stage: 4 for 2-bit (256 B per row, 30 KB of weights per stage),
+// 2 for 1.6-bit, whose larger activation slots would otherwise leave too few
+// stages in shared memory at M = 8.
+__host__ __device__ constexpr int gp_sg(int fmt) { return fmt == 2 ? 4 : 2; }
+__host__ __device__ constexpr int gp_stage_w(int fmt) { return gp_sg(fmt) * kGemvGroupBytes; }
+__host__ __device__ constexpr int gp_wbytes(int fmt) { return kGpRows * gp_stage_w(fmt); }
 constexpr int kGpMaxStages = 8;
 constexpr int kGpQueue = 32;                                  // items in flight per CTA
 constexpr int kGpPartBufs = 2;                                // consumer -> epilogue buffers
@@ -134,17 +138,17 @@ struct GpLayout {
         total;
     __host__ __device__ GpLayout(int fmt, int maxM) {
         const uint32_t group_bytes = fmt == 2 ? 512u : 640u;  // activations per token per group
-        raw_tok = kGpSG * group_bytes;                      // natural order, as copied
-        xtok = kGpSG * group_bytes + 64u;                   // staged token stride (bank offset)
+        raw_tok = gp_sg(fmt) * group_bytes;                 // natural order, as copied
+        xtok = gp_sg(fmt) * group_bytes + 64u;              // staged token stride (bank offset)
         raw_stage = (raw_tok * (uint32_t)maxM + 127u) & ~127u;
         x_stage = (xtok * (uint32_t)maxM + 127u) & ~127u;
-        const uint32_t per_stage = (uint32_t)kGpWBytes + raw_stage + x_stage;
+        const uint32_t per_stage = (uint32_t)gp_wbytes(fmt) + raw_stage + x_stage;
         const uint32_t fixed = (uint32_t)kGpPartBufs * kGpPartFloats * 4u +
                                kGpQueue * (uint32_t)sizeof(GpQEntry) +
                                8u * (3u * kGpMaxStages + 2u * kGpQueue + 2u * kGpPartBufs) + 256u;
         const uint32_t n = (kGpSmemBudget - fixed) / per_stage;
-        ns = n > (uint32_t)kGpMaxStages ? (uint32_t)kGpMaxStages : n;  // >= 5 for M <= 8
-        raw_off = ns * (uint32_t)kGpWBytes;
+        ns = n > (uint32_t)kGpMaxStages ? (uint32_t)kGpMaxStages : n;  // >= 3 for M <= 8
+        raw_off = ns * (uint32_t)gp_wbytes(fmt);
         x_off = raw_off + ns * raw_stage;
         part_off = x_off + ns * x_stage;
         q_off = part_off + (uint32_t)kGpPartBufs * kGpPartFloats * 4u;
@@ -157,6 +161,7 @@ struct GpItem {
     int l, tile, part, g0, g1;
 };
 
+template <int SG>
 __device__ __forceinline__ GpItem gp_decode(const GpArgs &a, int item) {
     int lo = 0, hi = a.count - 1;
     while (lo < hi) {
@@ -171,10 +176,10 @@ __device__ __forceinline__ GpItem gp_decode(const GpArgs &a, int item) {
     it.l = lo;
     it.tile = local / parts;
     it.part = local % parts;
-    // parts cut at stage (kGpSG-group) boundaries
-    const int stages = (groups + kGpSG - 1) / kGpSG;
-    it.g0 = kGpSG * (int)((int64_t)stages * it.part / parts);
-    it.g1 = min(groups, kGpSG * (int)((int64_t)stages * (it.part + 1) / parts));
+    // parts cut at stage (SG-group) boundaries
+    const int stages = (groups + SG - 1) / SG;
+    it.g0 = SG * (int)((int64_t)stages * it.part / parts);
+    it.g1 = min(groups, SG * (int)((int64_t)stages * (it.part + 1) / parts));
     return it;
 }
 
@@ -221,7 +226,10 @@ template <int FMT>
 __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_constant__ GpArgs a) {
     constexpr int TPB = FMT == 2 ? 4 : 5;
     constexpr int TRITS_GROUP = kGemvGroupBytes * TPB;  // 256 / 320 activations per group
-    constexpr int TRITS_STAGE = kGpSG * TRITS_GROUP;     // activations per token per stage
+    constexpr int SG = gp_sg(FMT);                       // K-groups per stage
+    constexpr int STAGE_W = gp_stage_w(FMT);             // weight bytes per row per stage
+    constexpr int WBYTES = gp_wbytes(FMT);               // weight bytes per stage
+    constexpr int TRITS_STAGE = SG * TRITS_GROUP;        // activations per token per stage
     constexpr int XUNITS = TRITS_STAGE / 8;              // 16-byte units per token per stage
     constexpr int GBYTES = G3X<FMT>::group_bytes;        // staged bytes per token per group
     constexpr uint32_t ONES = FMT == 2 ? 0x55555555u : 0x79797979u;  // every digit 1
@@ -254,7 +262,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         }
         for (int i = 0; i < kGpQueue; ++i) {
             mbar_init(&qfull[i], 1);
-            mbar_init(&qempty[i], kGpConsumers + 2);  // consumers, stager, epilogue
+            mbar_init(&qempty[i], kGpConsumers + 1 + kGpEpilogues);  // consumers, stager, epilogues
         }
         for (int i = 0; i < kGpPartBufs; ++i) {
             mbar_init(&pfull[i], kGpConsumers);
@@ -281,7 +289,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         GpItem it{};
         GpLayer L{};
         if (item < a.total_items) {
-            it = gp_decode(a, item);
+            it = gp_decode<SG>(a, item);
             L = a.L[it.l];
         }
         while (ok) {
@@ -319,7 +327,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             GpItem nit{};
             GpLayer NL{};
             if (next < a.total_items) {
-                nit = gp_decode(a, next);
+                nit = gp_decode<SG>(a, next);
                 NL = a.L[nit.l];
             }
             const CUtensorMap *tmap = a.maps + it.l;
@@ -360,15 +368,15 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             if (!waited) {
                 // first item: weights of up to a ring's worth of stages before the
                 // previous grid ends (expected bytes raised now, the arrival later)
-                const int nst = (it.g1 - it.g0 + kGpSG - 1) / kGpSG;
+                const int nst = (it.g1 - it.g0 + SG - 1) / SG;
                 const int pre = min(nst, NS);
                 if (lane == 0) {
                     tma_prefetch_desc(tmap);
                     for (int i = 0; i < pre; ++i) {
                         const int s = (int)((stage + i) % NS);
-                        mbar_expect_tx(&wfull[s], kGpWBytes);
-                        tma_load_2d(wring + s * kGpWBytes, tmap, &wfull[s],
-                                    (it.g0 + kGpSG * i) * kGemvGroupBytes, n0);
+                        mbar_expect_tx(&wfull[s], WBYTES);
+                        tma_load_2d(wring + s * WBYTES, tmap, &wfull[s],
+                                    (it.g0 + SG * i) * kGemvGroupBytes, n0);
                     }
                 }
                 pdl_wait();
@@ -378,14 +386,14 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 if (lane == 0) {
                     for (int i = 0; i < pre; ++i) {
                         const int s = (int)((stage + i) % NS);
-                        const int gi = it.g0 + kGpSG * i;
+                        const int gi = it.g0 + SG * i;
                         mbar_arrive_expect_tx(&wfull[s], deps ? (uint32_t)L.M * xbytes(gi) : 0u);
                         if (deps) issue_x(s, gi);
                     }
                 }
                 __syncwarp();
                 stage += pre;
-                g += kGpSG * pre;
+                g += SG * pre;
                 ps = pre;
                 if (ps == NS) { ps = 0; pph = 1; wrapped = true; }
                 if (!deps) { ok = false; break; }
@@ -393,7 +401,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 ok = false;
                 break;
             }
-            for (; g < it.g1; g += kGpSG, ++stage) {
+            for (; g < it.g1; g += SG, ++stage) {
                 const int s = ps;
                 if (wrapped && !warp_wait(&empty[s], pph ^ 1u)) {
                     ok = false;
@@ -405,8 +413,8 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                     wrapped = true;
                 }
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&wfull[s], kGpWBytes + (uint32_t)L.M * xbytes(g));
-                    tma_load_2d(wring + s * kGpWBytes, tmap, &wfull[s], g * kGemvGroupBytes, n0);
+                    mbar_arrive_expect_tx(&wfull[s], WBYTES + (uint32_t)L.M * xbytes(g));
+                    tma_load_2d(wring + s * WBYTES, tmap, &wfull[s], g * kGemvGroupBytes, n0);
                     issue_x(s, g);
                 }
                 __syncwarp();
@@ -429,7 +437,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         GpQEntry e;
         while (ok && gp_next_item(queue, qfull, qempty, qi, e)) {
             const int M = e.M, K = e.K;
-            for (int g = e.g0; g < e.g1; g += kGpSG) {
+            for (int g = e.g0; g < e.g1; g += SG) {
                 const int s = ss;
                 if (!warp_wait(&wfull[s], sph)) {
                     ok = false;
@@ -462,8 +470,8 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 if constexpr (FMT == 2) {
                     // natural order -> (x_i, x_{8+i}) pairs of each 16-activation word;
                     // item (token m, group h, lane chunk c, word j)
-                    for (int w = lane; w < M * 16 * kGpSG; w += 32) {
-                        const int m = w / (16 * kGpSG), r = w % (16 * kGpSG);
+                    for (int w = lane; w < M * 16 * SG; w += 32) {
+                        const int m = w / (16 * SG), r = w % (16 * SG);
                         const int h = r >> 4, c = (r >> 2) & 3, j = r & 3;
                         const int v0 = 32 * h + 8 * c + 2 * j;
                         const uint4 lo4 = load_unit(m, v0), hi4 = load_unit(m, v0 + 1);
@@ -492,12 +500,14 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 mbar_arrive(&xfull[s]);
             }
         }
-    } else if (warp == 2) {
-        // ---------------- epilogue ----------------
+    } else if (warp < 2 + kGpEpilogues) {
+        // ---------------- epilogues: warp 2 + i takes the items i, i + 2, ... ----------------
+        const int ew = warp - 2;
         pdl_wait();  // Y and the workspace may still be in use by the previous grid
-        int qi = 0, pi = 0;
+        int qi = 0, pi = -1;
         GpQEntry e;
         while (gp_next_item(queue, qfull, qempty, qi, e)) {
+            if (++pi % kGpEpilogues != ew) continue;  // another epilogue warp's item
             const int b = pi % kGpPartBufs;
             if (!warp_wait(&pfull[b], (uint32_t)(pi / kGpPartBufs) & 1u)) break;
             const float *pb = parts + b * kGpPartFloats;
@@ -518,7 +528,6 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&pempty[b]);
-            ++pi;
             bool final_tile = true;
             if (slot) {
                 __threadfence();
@@ -562,8 +571,9 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         }
     } else {
         // ---------------- consumers ----------------
-        const int cw = warp - 3;
-        const int rt = cw % kGpRowTiles, h = cw / kGpRowTiles;  // row tile, group of the stage
+        const int cw = warp - (2 + kGpEpilogues);
+        const int rt = cw % kGpRowTiles, hw = cw / kGpRowTiles;  // row tile, first group
+        constexpr int kHStep = kGpConsumers / kGpRowTiles;        // warps per row tile
         const int g = lane >> 2, c = lane & 3;
         const bool onesB = (g == 7);
         const int rowA = rt * kG3TileRows + g, rowB = rowA + 8;
@@ -577,7 +587,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             float acc[4][4], acc4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int q = 0; q < 4; ++q) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.f;
-            for (int gg = e.g0; gg < e.g1; gg += kGpSG) {
+            for (int gg = e.g0; gg < e.g1; gg += SG) {
                 const int s = cs;
                 if (!warp_wait(&wfull[s], cph) || !warp_wait(&xfull[s], cph)) {
                     ok = false;
@@ -587,11 +597,11 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                     cs = 0;
                     cph ^= 1u;
                 }
-                if (gg + h < e.g1) {  // this warp's group exists in the item
-                    const uint8_t *box = wring + s * kGpWBytes + h * kGemvGroupBytes + 16 * c;
-                    const uint4 wa = *reinterpret_cast<const uint4 *>(box + rowA * kGpStageW);
+                for (int h = hw; h < SG && gg + h < e.g1; h += kHStep) {  // groups of this warp
+                    const uint8_t *box = wring + s * WBYTES + h * kGemvGroupBytes + 16 * c;
+                    const uint4 wa = *reinterpret_cast<const uint4 *>(box + rowA * STAGE_W);
                     uint4 wb = make_uint4(ONES, ONES, ONES, ONES);
-                    if (!onesB) wb = *reinterpret_cast<const uint4 *>(box + rowB * kGpStageW);
+                    if (!onesB) wb = *reinterpret_cast<const uint4 *>(box + rowB * STAGE_W);
                     g3_group<FMT>(wa, wb, xs + s * lay.x_stage + tok * lay.xtok + h * GBYTES, c,
                                   lut_even, lut_odd, acc, acc4);
                 }
@@ -644,12 +654,13 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
 // ---- host side ---------------------------------------------------------------
 namespace tlk {
 
-// K-parts of a layer: items of about 8 K-groups (16 when M > 2, where each
-// split tile also writes and re-reads 120 x M partial sums); parts are cut at
-// stage boundaries, so there are at most as many parts as stages.
-inline int gp_parts(int groups, int M) {
-    const int target = M <= 2 ? 8 : 16;
-    const int stages = (groups + kGpSG - 1) / kGpSG;
+// K-parts of a layer: items of about eight stages (32 K-groups for 2-bit, 16
+// for 1.6-bit), so the per-item hand-offs stay small against the streaming;
+// parts are cut at stage boundaries, so there are at most as many parts as
+// stages.
+inline int gp_parts(int fmt, int groups, int M) {
+    const int target = 8 * gp_sg(fmt);
+    const int stages = (groups + gp_sg(fmt) - 1) / gp_sg(fmt);
     int parts = (groups + target / 2) / target;
     if (parts < 1) parts = 1;
     if (parts > stages) parts = stages;
@@ -693,7 +704,7 @@ inline GpSchedule gp_schedule(int fmt, int count, const GpHostLayer *in, GpLayer
         L.N = h.N;
         L.K = h.K;
         L.groups = (int)((rowbytes + kGemvGroupBytes - 1) / kGemvGroupBytes);
-        L.parts = gp_parts(L.groups, h.M);
+        L.parts = gp_parts(fmt, L.groups, h.M);
         L.tiles = (h.N + kGpRows - 1) / kGpRows;
         L.item_begin = sc.total_items;
         L.tile_begin = sc.total_tiles;
@@ -708,15 +719,15 @@ inline GpSchedule gp_schedule(int fmt, int count, const GpHostLayer *in, GpLayer
     return sc;
 }
 
-// Tensor map of a layer's packed weights: bytes x rows, boxes of 128 B x 120
-// rows (one stage), zero fill outside [0, row bytes) x [0, N).
+// Tensor map of a layer's packed weights: bytes x rows, boxes of one stage
+// (gp_stage_w bytes x 120 rows), zero fill outside [0, row bytes) x [0, N).
 inline bool gp_encode_map(int fmt, const GpHostLayer &h, CUtensorMap *map) {
     auto encode = tensor_map_encoder();
     if (!encode) return false;
     const int64_t rowbytes = fmt == 2 ? ((int64_t)h.K + 3) / 4 : ((int64_t)h.K + 4) / 5;
     cuuint64_t dims[2] = {(cuuint64_t)rowbytes, (cuuint64_t)h.N};
     cuuint64_t strides[1] = {(cuuint64_t)h.ldp};
-    cuuint32_t box[2] = {(cuuint32_t)kGpStageW, (cuuint32_t)kGpRows};
+    cuuint32_t box[2] = {(cuuint32_t)gp_stage_w(fmt), (cuuint32_t)kGpRows};
     cuuint32_t estr[2] = {1, 1};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(h.T), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
