@@ -12,31 +12,33 @@
 //
 // Work item = (layer, tile of 120 weight rows, K-part).  A layer's K-groups
 // (64 packed bytes per row each) are cut into `parts` contiguous ranges so
-// that items are all about the same size; items are claimed in order from a
-// counter in the caller's workspace (the first item of a CTA is its block
-// index, so its weights can be fetched before the previous grid finishes).
+// that items are all about the same size; CTA b of G takes the items b,
+// b + G, b + 2G, ... (its first item's weights are fetched before the
+// previous grid finishes, and the next item's record is loaded while the
+// current one streams).
 //
-// Every copy is a TMA copy: per K-group ("stage") one 2D tensor-map box of the
-// tile's 120 rows x 64 B (zero-filled past N and past the row), and one 1D bulk
-// copy per token of the activations at those K positions.  (Per-thread
+// Every copy is a TMA copy: per stage (gp_sg K-groups) one 2D tensor-map box
+// of the tile's 120 rows (zero-filled past N and past the row), and one 1D
+// bulk copy per token of the activations at those K positions.  (Per-thread
 // cp.async through L1 was measured at ~8-10 GB/s per SM here, far below the
 // ~40 GB/s per SM that HBM speed needs.)  The per-layer tensor maps and the
 // layer table live in the workspace, written once by tl_gemv_batch_plan.
 //
-// Warp roles of a CTA (640 threads):
+// Warp roles of a CTA (672 threads):
 //  * warp 0, producer: one elected lane issues each stage's copies into a ring
-//    of stages (completion counted in bytes on the stage's mbarrier), claims
-//    items and queues them for the other roles;
-//  * warp 1, stager: rewrites each stage's activations from natural order into
-//    the consumers' layout (2-bit: the pair order of the class-masked decode,
-//    see g3_word2; 1.6-bit: the interleaved units of gemv16_word), with zeros
-//    at k >= K;
-//  * warps 4..19, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
-//    rows and the all-ones row per warp; warps w and w + 8 take the two K-groups
-//    of each stage for the same rows), accumulating over the item's stages,
+//    of stages (completion counted in bytes on the stage's mbarrier) and
+//    queues the items for the other roles;
+//  * warps 1 and 2, stagers (alternate stages): rewrite each stage's
+//    activations from natural order into the consumers' layout (2-bit: the
+//    pair order of the class-masked decode, see g3_word2; 1.6-bit: the
+//    interleaved units of gemv16_word), with zeros at k >= K;
+//  * warps 5..20, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
+//    rows and the all-ones row per warp; the two warps of a row tile take
+//    alternate K-groups of each stage), accumulating over the item's stages,
 //    then handing the item's 2 x 120 x M sums to
-//  * warps 2 and 3, epilogues (alternate items): y = alpha * (sum - ones-row sum) to Y when the layer has
-//    one part; otherwise the part's fp32 partial goes to the workspace and the
+//  * warps 3 and 4, epilogues (alternate items): y = alpha * (sum - ones-row
+//    sum) to Y when the layer has one part; otherwise the part's fp32
+//    partial goes to the workspace and the
 //    last of the tile's parts to arrive (per-tile counter) adds the parts in
 //    part order (deterministic) and stores Y.  The tree reduction of per-warp
 //    partials through shared memory follows the Figure 11 caption text on
@@ -57,9 +59,12 @@ namespace tlk {
 
 constexpr int kGpRowTiles = 8;                               // 15-row tiles per item
 constexpr int kGpConsumers = 2 * kGpRowTiles;                 // two warps per row tile
+constexpr int kGpStagers = 2;                                 // stager warps (alternate stages)
 constexpr int kGpEpilogues = 2;                               // epilogue warps (alternate items)
-constexpr int kGpWarps = 2 + kGpEpilogues + kGpConsumers;    // + producer, stager
-constexpr int kGpThreads = 32 * kGpWarps;                    // 640
+constexpr int kGpFirstEpi = 1 + kGpStagers;                   // warp index of the first epilogue
+constexpr int kGpFirstCons = kGpFirstEpi + kGpEpilogues;      // warp index of the first consumer
+constexpr int kGpWarps = kGpFirstCons + kGpConsumers;
+constexpr int kGpThreads = 32 * kGpWarps;                    // 672
 constexpr int kGpRows = kGpRowTiles * kG3TileRows;            // 120 weight rows per item
 // K-groups per stage: 4 for 2-bit (256 B per row, 30 KB of weights per stage),
 // 2 for 1.6-bit, whose larger activation slots would otherwise leave too few
@@ -94,7 +99,7 @@ struct GpLayer {
 };
 
 // Workspace layout of a planned batch (every region 256-byte aligned):
-//   header  : kGpHeaderWords u32 counters: [1] final tiles, [2] CTAs done
+//   header  : kGpHeaderWords u32 counters: [1] final tiles, [2] CTAs done ([0] unused)
 //   layers  : count x GpLayer
 //   maps    : count x CUtensorMap (the packed weights of each layer)
 //   tiles   : total_tiles x u32, parts of each tile that have arrived
@@ -262,7 +267,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         }
         for (int i = 0; i < kGpQueue; ++i) {
             mbar_init(&qfull[i], 1);
-            mbar_init(&qempty[i], kGpConsumers + 1 + kGpEpilogues);  // consumers, stager, epilogues
+            mbar_init(&qempty[i], kGpConsumers + kGpStagers + kGpEpilogues);
         }
         for (int i = 0; i < kGpPartBufs; ++i) {
             mbar_init(&pfull[i], kGpConsumers);
@@ -428,8 +433,10 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         // the CTA may not exit with copies still landing in its shared memory
         for (uint32_t t = stage > (uint32_t)NS ? stage - NS : 0; t < stage; ++t)
             mbar_wait(&wfull[t % NS], (t / NS) & 1u);
-    } else if (warp == 1) {
-        // ---------------- stager ----------------
+    } else if (warp < kGpFirstEpi) {
+        // ---------------- stagers: warp 1 + i takes the stages i, i + 2, ... ----------------
+        const uint32_t sw = (uint32_t)(warp - 1);
+        uint32_t st = 0;  // running stage index
         int ss = 0;
         uint32_t sph = 0;
         int qi = 0;
@@ -439,13 +446,15 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             const int M = e.M, K = e.K;
             for (int g = e.g0; g < e.g1; g += SG) {
                 const int s = ss;
-                if (!warp_wait(&wfull[s], sph)) {
-                    ok = false;
-                    break;
-                }
+                const uint32_t ph = sph;
                 if (++ss == NS) {
                     ss = 0;
                     sph ^= 1u;
+                }
+                if ((st++ % kGpStagers) != sw) continue;  // the other stager's stage
+                if (!warp_wait(&wfull[s], ph)) {
+                    ok = false;
+                    break;
                 }
                 // activations of this stage below K (and below the item's last group)
                 const int valid = min(K - g * TRITS_GROUP, (e.g1 - g) * TRITS_GROUP);
@@ -500,9 +509,9 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                 mbar_arrive(&xfull[s]);
             }
         }
-    } else if (warp < 2 + kGpEpilogues) {
-        // ---------------- epilogues: warp 2 + i takes the items i, i + 2, ... ----------------
-        const int ew = warp - 2;
+    } else if (warp < kGpFirstCons) {
+        // ---------------- epilogues: warp 3 + i takes the items i, i + 2, ... ----------------
+        const int ew = warp - kGpFirstEpi;
         pdl_wait();  // Y and the workspace may still be in use by the previous grid
         int qi = 0, pi = -1;
         GpQEntry e;
@@ -571,7 +580,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         }
     } else {
         // ---------------- consumers ----------------
-        const int cw = warp - (2 + kGpEpilogues);
+        const int cw = warp - kGpFirstCons;
         const int rt = cw % kGpRowTiles, hw = cw / kGpRowTiles;  // row tile, first group
         constexpr int kHStep = kGpConsumers / kGpRowTiles;        // warps per row tile
         const int g = lane >> 2, c = lane & 3;
