@@ -24,19 +24,20 @@
 // ~40 GB/s per SM that HBM speed needs.)  The per-layer tensor maps and the
 // layer table live in the workspace, written once by tl_gemv_batch_plan.
 //
-// Warp roles of a CTA (672 threads):
+// Warp roles of a CTA (704 threads):
 //  * warp 0, producer: one elected lane issues each stage's copies into a ring
 //    of stages (completion counted in bytes on the stage's mbarrier) and
 //    queues the items for the other roles;
-//  * warps 1 and 2, stagers (alternate stages): rewrite each stage's
-//    activations from natural order into the consumers' layout (2-bit: the
+//  * warps 1..3, stagers (warp 1 + i owns the ring slots s with s mod 3 = i):
+//    rewrite each stage's activations from natural order into the consumers'
+//    layout (2-bit: the
 //    pair order of the class-masked decode, see g3_word2; 1.6-bit: the
 //    interleaved units of gemv16_word), with zeros at k >= K;
-//  * warps 5..20, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
+//  * warps 6..21, consumers: the decode + mma.sync of tl_gemv3.cuh (15 weight
 //    rows and the all-ones row per warp; the two warps of a row tile take
 //    alternate K-groups of each stage), accumulating over the item's stages,
 //    then handing the item's 2 x 120 x M sums to
-//  * warps 3 and 4, epilogues (alternate items): y = alpha * (sum - ones-row
+//  * warps 4 and 5, epilogues (alternate items): y = alpha * (sum - ones-row
 //    sum) to Y when the layer has one part; otherwise the part's fp32
 //    partial goes to the workspace and the
 //    last of the tile's parts to arrive (per-tile counter) adds the parts in
@@ -59,12 +60,12 @@ namespace tlk {
 
 constexpr int kGpRowTiles = 8;                               // 15-row tiles per item
 constexpr int kGpConsumers = 2 * kGpRowTiles;                 // two warps per row tile
-constexpr int kGpStagers = 2;                                 // stager warps (alternate stages)
+constexpr int kGpStagers = 3;                                 // stager warps (each owns ring slots)
 constexpr int kGpEpilogues = 2;                               // epilogue warps (alternate items)
 constexpr int kGpFirstEpi = 1 + kGpStagers;                   // warp index of the first epilogue
 constexpr int kGpFirstCons = kGpFirstEpi + kGpEpilogues;      // warp index of the first consumer
 constexpr int kGpWarps = kGpFirstCons + kGpConsumers;
-constexpr int kGpThreads = 32 * kGpWarps;                    // 672
+constexpr int kGpThreads = 32 * kGpWarps;                    // 704
 constexpr int kGpRows = kGpRowTiles * kG3TileRows;            // 120 weight rows per item
 // K-groups per stage: 4 for 2-bit (256 B per row, 30 KB of weights per stage),
 // 2 for 1.6-bit, whose larger activation slots would otherwise leave too few
@@ -434,9 +435,10 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
         for (uint32_t t = stage > (uint32_t)NS ? stage - NS : 0; t < stage; ++t)
             mbar_wait(&wfull[t % NS], (t / NS) & 1u);
     } else if (warp < kGpFirstEpi) {
-        // ---------------- stagers: warp 1 + i takes the stages i, i + 2, ... ----------------
-        const uint32_t sw = (uint32_t)(warp - 1);
-        uint32_t st = 0;  // running stage index
+        // ---------------- stagers: warp 1 + i takes the ring slots s with s % kGpStagers == i ----
+        // (owning slots, not every k-th stage: a stager then waits every round of
+        // its slots in order, so a parity wait never sees a phase two rounds back)
+        const int sw = warp - 1;
         int ss = 0;
         uint32_t sph = 0;
         int qi = 0;
@@ -451,7 +453,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
                     ss = 0;
                     sph ^= 1u;
                 }
-                if ((st++ % kGpStagers) != sw) continue;  // the other stager's stage
+                if (s % kGpStagers != sw) continue;  // another stager's slot
                 if (!warp_wait(&wfull[s], ph)) {
                     ok = false;
                     break;
@@ -510,7 +512,7 @@ __global__ void __launch_bounds__(kGpThreads, 1) gemvp_kernel(const __grid_const
             }
         }
     } else if (warp < kGpFirstCons) {
-        // ---------------- epilogues: warp 3 + i takes the items i, i + 2, ... ----------------
+        // ---------------- epilogues: warp 4 + i takes the items i, i + 2, ... ----------------
         const int ew = warp - kGpFirstEpi;
         pdl_wait();  // Y and the workspace may still be in use by the previous grid
         int qi = 0, pi = -1;

@@ -73,6 +73,29 @@ def _counters_zero(ws):
 MIXED = [(1, 1, 1, 1 / 3), (3, 7, 5, 0.2), (8, 121, 255, 0.6), (2, 250, 257, 1 / 3),
          (1, 240, 1000, 1 / 3), (5, 130, 2049, 0.2), (1, 300, 4100, 1 / 3), (8, 64, 14336, 1 / 3),
          (1, 1000, 3072, 0.6), (4, 129, 8200, 1 / 3)]
+# short batches whose M = 8 layer has a partial last stage and wraps the ring
+SHORT = [[(1, 500, 3000), (8, 130, 4100), (3, 77, 700)], [(8, 130, 4100)],
+         [(8, 250, 4100), (8, 130, 1025)]]
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+@pytest.mark.parametrize("shapes", SHORT)
+def test_short_batches(fmt, shapes):
+    import ternary_weight_03_b200 as tl
+    cases, specs = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        T = synth.trits(700 + i, N, K)
+        X = synth.activations(710 + i, M, K)
+        a = synth.alpha_for(720 + i)
+        dP, dX, dY = _device_layer(fmt, T, X)
+        cases.append((T, X, a, dY, N, M))
+        specs.append((dP, a, dX, K, dY))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    tl.gemv_batch_run(plan)
+    assert tl.device_status() == 0
+    for T, X, a, dY, N, M in cases:
+        _check_layer(T, X, a, dY, N, M)
 
 
 @pytest.mark.parametrize("fmt", [2, 16])
