@@ -282,3 +282,40 @@ def test_long_chain_multiple_items_per_cta(fmt):
             tol = tol + abs(alphas[i]) * ulp.sum(axis=1)[:, None]
         assert (np.abs(got - ref) <= tol).all(), f"layer {i}"
         x = ys[i].cpu().numpy()
+
+
+DECODE_LAYER = [(3072, 3072)] * 4 + [(3072, 8192)] * 2 + [(8192, 3072)]  # q k v o gate up down
+
+
+@pytest.mark.parametrize("fmt,M", [(2, 1), (2, 8), (16, 1)])
+def test_decode_step_210_layers_sampled(fmt, M):
+    """The 30-layer decode step (210 matrices, 849 MB packed at 2 bits) as ONE
+    batch launch, the configuration the bench times; per layer, sampled
+    outputs against the oracle computed one by one (trits regenerated from
+    their seeds for the check, so host memory stays at one layer)."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    mats = [(K, N, 1000 + 7 * layer + j) for layer in range(30)
+            for j, (K, N) in enumerate(DECODE_LAYER)]
+    specs, xs = [], []
+    for (K, N, seed) in mats:
+        P = tl.pack(fmt, synth.trits(seed, N, K))
+        X = synth.activations(seed, M, K)
+        xs.append(X)
+        specs.append((torch.from_numpy(P).cuda(), synth.alpha_for(seed), torch.from_numpy(X).cuda(),
+                      K, torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+    assert tl.device_status() == 0
+    o = oracle.get()
+    rng = np.random.default_rng(fmt * 10 + M)
+    for (K, N, seed), X, sp in zip(mats, xs, specs):
+        Y = sp[4].float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(Y).all()
+        T = synth.trits(seed, N, K)
+        ms = np.concatenate([rng.integers(0, M, 24), [M - 1]])
+        ns = np.concatenate([rng.integers(0, N, 24), [N - 1]])
+        ref = o.linear_at(T, X, sp[1], ms, ns)
+        tol = oracle.tolerance(ref, X[ms], sp[1])
+        assert (np.abs(Y[ms, ns] - ref) <= tol).all(), f"layer seed {seed}"
