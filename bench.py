@@ -492,37 +492,40 @@ def secondary(dev, stream, quick: bool):
                                 "ms_per_step": round(ms / 5, 4)}
     del sw
     torch.cuda.empty_cache()
-    # batched GEMM
-    gemm = {}
-    for (K, N) in ((4096, 14336), (14336, 4096)):
-        P, _, alpha = make_matrix(2, K, N, 0)
-        dP = torch.from_numpy(P).to(dev)
-        for M in ((16, 256, 4096) if quick else (16, 64, 256, 1024, 4096)):
-            import synth
-            X = torch.from_numpy(synth.activations(1, M, K)).to(dev)
-            Y = torch.empty((M, N), dtype=torch.float16, device=dev)
-            rc = tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
-                                  Y.data_ptr(), N, M, N, K, stream.cuda_stream)
-            if rc != 0:
-                gemm[f"M{M}_K{K}_N{N}"] = {"status": tl.status_str(rc)}
-                continue
-            with torch.cuda.stream(stream):
-                for _ in range(3):
-                    tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
-                                     Y.data_ptr(), N, M, N, K, stream.cuda_stream)
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                reps = 10
-                a.record(stream)
-                for _ in range(reps):
-                    tl.lib().tl_gemm(2, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(), K,
-                                     Y.data_ptr(), N, M, N, K, stream.cuda_stream)
-                b.record(stream)
-                torch.cuda.synchronize()
-            us = a.elapsed_time(b) * 1e3 / reps
-            tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
-            gemm[f"M{M}_K{K}_N{N}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 1),
-                                       "frac_tensor": round(tf / pk["bf16_tflops"], 4)}
-    out["gemm_2bit"] = gemm
+    # batched GEMM, both formats
+    import synth
+    for fmt, key in ((2, "gemm_2bit"), (16, "gemm_1p6bit")):
+        gemm = {}
+        for (K, N) in ((4096, 14336), (14336, 4096)):
+            P, _, alpha = make_matrix(fmt, K, N, 0)
+            dP = torch.from_numpy(P).to(dev)
+            for M in ((16, 256, 4096) if quick else (16, 64, 256, 1024, 4096)):
+                X = torch.from_numpy(synth.activations(1, M, K)).to(dev)
+                Y = torch.empty((M, N), dtype=torch.float16, device=dev)
+
+                def call():
+                    return tl.lib().tl_gemm(fmt, dP.data_ptr(), dP.stride(0), alpha, X.data_ptr(),
+                                            K, Y.data_ptr(), N, M, N, K, stream.cuda_stream)
+                rc = call()
+                if rc != 0:
+                    gemm[f"M{M}_K{K}_N{N}"] = {"status": tl.status_str(rc)}
+                    continue
+                with torch.cuda.stream(stream):
+                    for _ in range(3):
+                        call()
+                    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    reps = 10
+                    a.record(stream)
+                    for _ in range(reps):
+                        call()
+                    b.record(stream)
+                    torch.cuda.synchronize()
+                us = a.elapsed_time(b) * 1e3 / reps
+                tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+                gemm[f"M{M}_K{K}_N{N}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 1),
+                                           "frac_tensor": round(tf / pk["bf16_tflops"], 4)}
+            del dP
+        out[key] = gemm
     out["decode_step_30_layers"] = decode_step(dev, stream)
     # the same 2-bit sweep as twelve tl_gemv_ex calls per step (with and without PDL)
     sw = Sweep(2, dev)

@@ -223,8 +223,12 @@ int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream);
 
 /* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and
- * rules as tl_gemv (tensor-core kernel: packed tiles are expanded to fp16
- * on chip and multiplied with tcgen05 MMAs accumulating in fp32). */
+ * rules as tl_gemv, both formats ("Pith review of Spectra 1.1", "What carries
+ * the argument": an FP16 x INT2 tensor-core kernel with fused dequantisation;
+ * the 1.6-bit packing of "Core claim" goes through the same kernel).  Packed
+ * tiles are expanded on chip to exact fp16 -1 / 0 / +1 and multiplied with
+ * tcgen05 MMAs accumulating in fp32.  For a given format and shape the
+ * summation order is fixed, so repeated calls agree bit for bit. */
 int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
             int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream);
 

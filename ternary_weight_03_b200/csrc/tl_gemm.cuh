@@ -1,14 +1,17 @@
 // tl_gemm.cuh -- batched / prefill ternary linear layer, M >= 16:
 //   Y[m][n] = fp16_rn(alpha * sum_k T[n][k] * X[m][k])
-// on the sm_100a tensor cores (tcgen05, fp32 accumulators in tensor memory).
+// on the sm_100a tensor cores (tcgen05, fp32 accumulators in tensor memory),
+// for both storage formats (2-bit base 4 and 1.6-bit base 3).
 //
 // The pages' GPU kernel is an FP16 x INT2 tensor-core kernel with
 // asynchronous copies and fused dequantisation ("Pith review of Spectra
 // 1.1", "What carries the argument").  Here, per CTA and output tile of
 // 128 weight rows x BN tokens:
-//  * a TMA warp streams, per K-step of 64, the packed tile (128 rows x 16 B)
-//    and the activation tile (BN tokens x 64 fp16, 128-byte swizzle) into a
-//    shared-memory ring (no multicast);
+//  * a TMA warp streams, per K-step of 64, the activation tile (BN tokens x
+//    64 fp16, 128-byte swizzle) and, for the 2-bit format, the packed tile
+//    (128 rows x 16 B) into a shared-memory ring (no multicast).  A 1.6-bit
+//    row holds 64 trits in 12.8 bytes, so its packed tiles come in blocks of
+//    320 trits (128 rows x 64 B, five K-steps) through a separate 2-deep ring;
 //  * four decode warps (thread = weight row = TMEM lane) expand the row's 64
 //    trits to exact fp16 -1 / 0 / +1 and write them with tcgen05.st straight
 //    into tensor memory, where they are the MMA's A operand -- the expanded
@@ -19,7 +22,8 @@
 //  * the decode warps then read the accumulator with tcgen05.ld, scale by
 //    alpha and store fp16.
 // Split-K, for shapes with fewer output tiles than SMs: a cluster of S CTAs
-// shares one output tile, rank r taking K-steps [r nk / S, (r + 1) nk / S).
+// shares one output tile, rank r taking K-steps [r nk / S, (r + 1) nk / S)
+// (1.6-bit: whole 320-trit blocks, so every rank starts on a block).
 // After one cluster barrier (every ring is then idle), the accumulator is
 // cut into units of 32 rows (a TMEM lane quarter) x 32 columns; unit u is
 // owned by rank u mod S.  Each CTA pushes the units it does not own from
@@ -47,10 +51,18 @@ __host__ __device__ constexpr int gemm_tmem_cols(int bn) {
     return gemm_acol_base(bn) + 32 * 4 <= 256 ? 256 : 512;
 }
 
+template <int FMT>
 struct GemmSmem {
-    // per-stage byte offsets inside the dynamic shared memory block
+    // per-stage byte sizes inside the dynamic shared memory block
     __host__ __device__ static constexpr uint32_t x_stage_bytes(int bn) { return (uint32_t)bn * 128u; }
-    static constexpr uint32_t w_stage_bytes = kGemmRows * 16u;
+    // 2-bit: one packed tile (128 rows x 16 B = 64 trits) per K-step, filled
+    // with the activation stage of the same K-step.  1.6-bit: 64 trits are
+    // 12.8 bytes, so packed tiles come in blocks of 320 trits (128 rows x 64 B,
+    // five K-steps) through a 2-deep ring of their own.
+    static constexpr uint32_t w_row_bytes = FMT == 2 ? 16u : 64u;
+    static constexpr uint32_t w_stage_bytes = kGemmRows * w_row_bytes;
+    static constexpr int w_stages = FMT == 2 ? kGemmStages : 2;
+    static constexpr int ksteps_per_w = FMT == 2 ? 1 : 5;
 };
 
 // Exact decode of one 32-bit word of 2-bit digits (16 trits, natural order)
@@ -72,30 +84,90 @@ __device__ __forceinline__ void decode2_exact(uint32_t w, uint32_t *out) {
     }
 }
 
-template <int BN>
+// Base-3 digits of the four bytes of w (byte = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4):
+// E[i] holds digit i of byte b in its byte lane b.  The bytes are spread over
+// two registers of 16-bit lanes; for v <= 255, floor(v / 3) = (v * 171) >> 9
+// and v * 171 < 2^16, so both lanes divide at once without a carry between them.
+__device__ __forceinline__ void digits3_word(uint32_t w, uint32_t (&E)[5]) {
+    uint32_t lo = w & 0x00FF00FFu;         // bytes 0 and 2
+    uint32_t hi = (w >> 8) & 0x00FF00FFu;  // bytes 1 and 3
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t qlo = ((lo * 171u) >> 9) & 0x007F007Fu;
+        const uint32_t qhi = ((hi * 171u) >> 9) & 0x007F007Fu;
+        E[i] = (lo - 3u * qlo) | ((hi - 3u * qhi) << 8);  // v mod 3, lane by lane
+        lo = qlo;
+        hi = qhi;
+    }
+    E[4] = lo | (hi << 8);
+}
+
+// Exact decode of K-step J (trits 64 J .. 64 J + 63) of a 320-trit block of
+// 1.6-bit codes (64 bytes in w[0..15]; trit 5 b + i is digit i of byte b) into
+// 32 fp16x2 registers (t_2c, t_2c+1), values -1, 0, +1.  Once the loops
+// unroll, every word, digit and byte index below is a compile-time constant.
+template <int J>
+__device__ __forceinline__ void decode16_kstep(const uint32_t (&w)[16], uint32_t (&out)[32]) {
+    constexpr int kW0 = (64 * J / 5) / 4, kW1 = ((64 * J + 63) / 5) / 4;
+    uint32_t E[kW1 - kW0 + 1][5];
+#pragma unroll
+    for (int q = 0; q <= kW1 - kW0; ++q) digits3_word(w[kW0 + q], E[q]);
+    const __half2 off = __halves2half2(__ushort_as_half(0x6401), __ushort_as_half(0x6401));
+#pragma unroll
+    for (int c = 0; c < 32; ++c) {
+        const int t0 = 64 * J + 2 * c, t1 = t0 + 1;
+        const int b0 = t0 / 5, b1 = t1 / 5;
+        // result bytes: digit of t0, 0x00 (sign of a digit byte), digit of t1, 0x00
+        const uint32_t sel =
+            (uint32_t)(b0 & 3) | 0x80u | ((uint32_t)(4 + (b1 & 3)) << 8) | 0x8000u;
+        uint32_t p = prmt(E[b0 / 4 - kW0][t0 % 5], E[b1 / 4 - kW0][t1 % 5], sel) | 0x64006400u;
+        __half2 h = __hsub2(*reinterpret_cast<__half2 *>(&p), off);  // 1024 + d - 1025 = t
+        out[c] = *reinterpret_cast<uint32_t *>(&h);
+    }
+}
+
+__device__ __forceinline__ void decode16_kstep(int j, const uint32_t (&w)[16], uint32_t (&out)[32]) {
+    switch (j) {
+        case 0: decode16_kstep<0>(w, out); break;
+        case 1: decode16_kstep<1>(w, out); break;
+        case 2: decode16_kstep<2>(w, out); break;
+        case 3: decode16_kstep<3>(w, out); break;
+        default: decode16_kstep<4>(w, out); break;
+    }
+}
+
+template <int FMT, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-             float alpha, uint16_t *__restrict__ Y, int64_t ldy, int M, int N, int K) {
+gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+            float alpha, uint16_t *__restrict__ Y, int64_t ldy, int M, int N, int K) {
+    using L = GemmSmem<FMT>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled activation stages
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *xs = smem;                                            // kGemmStages x BN x 128 B
-    uint8_t *ws = xs + kGemmStages * GemmSmem::x_stage_bytes(BN);  // kGemmStages x 128 x 16 B
-    uint64_t *full = reinterpret_cast<uint64_t *>(ws + kGemmStages * GemmSmem::w_stage_bytes);
+    uint8_t *xs = smem;                                         // kGemmStages x BN x 128 B
+    uint8_t *ws = xs + kGemmStages * L::x_stage_bytes(BN);      // w_stages x 128 x w_row_bytes
+    uint64_t *full = reinterpret_cast<uint64_t *>(ws + L::w_stages * L::w_stage_bytes);
     uint64_t *afull = full + kGemmStages;   // decoders -> MMA (A stage written)
     uint64_t *empty = afull + kGemmStages;  // MMA commit -> producer / decoders
     uint64_t *done = empty + kGemmStages;   // last MMA committed -> epilogue
     uint64_t *redbar = done + 1;            // split-K: the partials pushed to this CTA landed
-    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(redbar + 1);
+    uint64_t *wfull = redbar + 1;           // 1.6-bit: packed block landed
+    uint64_t *wempty = wfull + 2;           // 1.6-bit: packed block read by all 128 decoders
+    uint32_t *tmem_base_slot = reinterpret_cast<uint32_t *>(wempty + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n0 = blockIdx.x * kGemmRows;
     const int m0 = blockIdx.y * BN;
     const int nk_all = (K + kGemmKStep - 1) / kGemmKStep;
-    // split-K rank and K-step range (the host keeps S <= nk_all, so no range is empty)
+    // split-K rank and K-step range, cut in units of KU K-steps (one packed
+    // block) so that every rank starts on a block; the host keeps S <= the
+    // number of units, so no range is empty
+    constexpr int KU = L::ksteps_per_w;
     const uint32_t S = cluster_nctarank(), rank = cluster_ctarank();
-    const int kb = (int)(((int64_t)nk_all * rank) / S);
-    const int nk = (int)(((int64_t)nk_all * (rank + 1)) / S) - kb;
+    const int nu = (nk_all + KU - 1) / KU;
+    const int kb = KU * (int)(((int64_t)nu * rank) / S);
+    const int ke = min(nk_all, KU * (int)(((int64_t)nu * (rank + 1)) / S));
+    const int nk = ke - kb;
     // accumulator units: 4 lane quarters x kChunks column chunks of kChunkW
     constexpr int kChunkW = BN < 32 ? BN : 32;
     constexpr int kChunks = (BN + 31) / 32;
@@ -108,6 +180,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         }
         mbar_init(done, 1);
         mbar_init(redbar, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&wfull[s], 1);
+            mbar_init(&wempty[s], 128);
+        }
         // bytes pushed here: (S - 1) sources x the tile's 128 x BN floats / S
         if (S > 1) mbar_arrive_expect_tx(redbar, (S - 1) * (uint32_t)(kGemmRows * BN * 4) / S);
         fence_mbar_init();
@@ -126,22 +202,33 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
     if (warp == 0) {
         // ---- TMA producer ----
         if (lane == 0) {
-            const uint32_t bytes = GemmSmem::x_stage_bytes(BN) + GemmSmem::w_stage_bytes;
+            const uint32_t bytes = L::x_stage_bytes(BN) + (FMT == 2 ? L::w_stage_bytes : 0u);
+            int issued = 0, wissued = 0;
             for (int k = 0; k < nk; ++k) {
                 const int s = k % kGemmStages;
                 if (k >= kGemmStages && !mbar_wait(&empty[s], ((k / kGemmStages) - 1) & 1))
                     break;
+                if (FMT != 2 && k % KU == 0) {
+                    // next packed block, once all decoders have read the one two back
+                    const int b = k / KU, wsl = b & 1;
+                    if (b >= 2 && !mbar_wait(&wempty[wsl], ((b >> 1) - 1) & 1)) break;
+                    mbar_arrive_expect_tx(&wfull[wsl], L::w_stage_bytes);
+                    tma_load_2d(ws + wsl * L::w_stage_bytes, &tmap_w, &wfull[wsl],
+                                (kb / KU + b) * (int)L::w_row_bytes, n0);
+                    wissued = b + 1;
+                }
                 mbar_arrive_expect_tx(&full[s], bytes);
-                tma_load_2d(xs + s * GemmSmem::x_stage_bytes(BN), &tmap_x, &full[s],
+                tma_load_2d(xs + s * L::x_stage_bytes(BN), &tmap_x, &full[s],
                             (kb + k) * kGemmKStep, m0);
-                tma_load_2d(ws + s * GemmSmem::w_stage_bytes, &tmap_w, &full[s], (kb + k) * 16,
-                            n0);
+                if (FMT == 2)
+                    tma_load_2d(ws + s * L::w_stage_bytes, &tmap_w, &full[s], (kb + k) * 16, n0);
+                issued = k + 1;
             }
             // drain: make sure every issued copy has landed before the CTA may exit
-            for (int k = nk - kGemmStages > 0 ? nk - kGemmStages : 0; k < nk; ++k) {
-                const int s = k % kGemmStages;
-                mbar_wait(&full[s], (k / kGemmStages) & 1);
-            }
+            for (int k = issued > kGemmStages ? issued - kGemmStages : 0; k < issued; ++k)
+                mbar_wait(&full[k % kGemmStages], (k / kGemmStages) & 1);
+            for (int b = wissued > 2 ? wissued - 2 : 0; b < wissued; ++b)
+                mbar_wait(&wfull[b & 1], (b >> 1) & 1);
         }
     } else if (warp == 1) {
         // ---- MMA issuer ----
@@ -149,13 +236,13 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
             constexpr uint32_t idesc = idesc_f16_f32(kGemmRows, BN);
             for (int k = 0; k < nk; ++k) {
                 const int s = k % kGemmStages;
-                // the decoders saw this stage's TMA complete before arriving; wait on
-                // it here too so the tensor core's reads are ordered after the copy
+                // the activation stage has landed and the decoders wrote A stage s
+                // (2-bit: after seeing the same copy complete)
                 if (!mbar_wait(&full[s], (k / kGemmStages) & 1) ||
                     !mbar_wait(&afull[s], (k / kGemmStages) & 1))
                     break;
                 tc_fence_after();
-                const uint32_t xaddr = smem_u32(xs + s * GemmSmem::x_stage_bytes(BN));
+                const uint32_t xaddr = smem_u32(xs + s * L::x_stage_bytes(BN));
 #pragma unroll
                 for (int j = 0; j < kGemmKStep / 16; ++j) {
                     const uint64_t bdesc = sdesc_k128(xaddr + 32 * j);
@@ -172,21 +259,49 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
         const int row = quarter * 32 + lane;      // row within the tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
+        uint32_t blk[16];  // 1.6-bit: this row's current 320-trit block
         for (int k = 0; k < nk && ok; ++k) {
             const int s = k % kGemmStages;
-            ok = mbar_wait(&full[s], (k / kGemmStages) & 1);
-            if (ok && k >= kGemmStages) ok = mbar_wait(&empty[s], ((k / kGemmStages) - 1) & 1);
-            if (!ok) break;
-            const uint4 pw = *reinterpret_cast<const uint4 *>(ws + s * GemmSmem::w_stage_bytes +
-                                                               row * 16);
             uint32_t a[32];
-            decode2_exact(pw.x, a);
-            decode2_exact(pw.y, a + 8);
-            decode2_exact(pw.z, a + 16);
-            decode2_exact(pw.w, a + 24);
-            // the packed bytes are consumed; order these generic reads before the
-            // TMA write that will refill this stage once the MMA releases it
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            if constexpr (FMT == 2) {
+                ok = mbar_wait(&full[s], (k / kGemmStages) & 1);
+                if (ok && k >= kGemmStages) ok = mbar_wait(&empty[s], ((k / kGemmStages) - 1) & 1);
+                if (!ok) break;
+                const uint4 pw = *reinterpret_cast<const uint4 *>(ws + s * L::w_stage_bytes +
+                                                                   row * 16);
+                decode2_exact(pw.x, a);
+                decode2_exact(pw.y, a + 8);
+                decode2_exact(pw.z, a + 16);
+                decode2_exact(pw.w, a + 24);
+                // the packed bytes are consumed; order these generic reads before the
+                // TMA write that will refill this stage once the MMA releases it
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            } else {
+                const int j = k % KU;
+                if (j == 0) {
+                    const int b = k / KU, wsl = b & 1;
+                    ok = mbar_wait(&wfull[wsl], (b >> 1) & 1);
+                    if (!ok) break;
+                    const uint4 *src = reinterpret_cast<const uint4 *>(
+                        ws + wsl * L::w_stage_bytes + row * L::w_row_bytes);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = src[q];
+                        blk[4 * q] = v.x;
+                        blk[4 * q + 1] = v.y;
+                        blk[4 * q + 2] = v.z;
+                        blk[4 * q + 3] = v.w;
+                    }
+                    // order the generic reads before the TMA write that refills the slot
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    mbar_arrive(&wempty[wsl]);
+                }
+                if (k >= kGemmStages && !mbar_wait(&empty[s], ((k / kGemmStages) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                decode16_kstep(j, blk, a);
+            }
             tc_fence_after();
             tmem_st_32x32b_x32(tmem + lane_addr + gemm_acol_base(BN) + 32 * s, a);
             tc_wait_st();
@@ -305,21 +420,23 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__
 
 // ---- host side ---------------------------------------------------------------
 // Every CTA asks for more than half of an SM's 228 KB of shared memory, so at
-// most one CTA of this kernel (of any BN, from any number of concurrent
-// launches) is resident per SM and its TMEM allocation (<= 512 columns) never
-// waits.  tcgen05.alloc blocks while columns are taken; with split-K clusters
-// such a wait could close a cycle (a CTA holding TMEM at the cluster barrier
-// for a peer that waits for TMEM behind it).
+// most one CTA of this kernel (of any format or BN, from any number of
+// concurrent launches) is resident per SM and its TMEM allocation (<= 512
+// columns) never waits.  tcgen05.alloc blocks while columns are taken; with
+// split-K clusters such a wait could close a cycle (a CTA holding TMEM at the
+// cluster barrier for a peer that waits for TMEM behind it).
 constexpr size_t kGemmMinSmem = 116 * 1024 + 1;
+template <int FMT>
 inline size_t gemm_smem_bytes(int bn) {
-    const size_t need = 1024 + kGemmStages * ((size_t)bn * 128 + kGemmRows * 16) +
-                        (3 * kGemmStages + 2) * 8 + 16;
+    using L = GemmSmem<FMT>;
+    const size_t need = 1024 + kGemmStages * (size_t)L::x_stage_bytes(bn) +
+                        (size_t)L::w_stages * L::w_stage_bytes + (3 * kGemmStages + 6) * 8 + 16;
     return need > kGemmMinSmem ? need : kGemmMinSmem;
 }
 
-// CTAs of gemm2_kernel<BN> that can be resident at once in clusters of S
+// CTAs of gemm_kernel<FMT, BN> that can be resident at once in clusters of S
 // (cached per device and S; -1 if the occupancy query fails).
-template <int BN>
+template <int FMT, int BN>
 inline int gemm_resident(int dev, int S, size_t smem) {
     constexpr int kMaxDev = 64;
     static std::mutex mu;
@@ -342,7 +459,8 @@ inline int gemm_resident(int dev, int S, size_t smem) {
     q.attrs = at;
     q.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm2_kernel<BN>, &q) != cudaSuccess) return -1;
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_kernel<FMT, BN>, &q) != cudaSuccess)
+        return -1;
     std::lock_guard<std::mutex> lock(mu);
     cache[dev][si] = clusters * S > 0 ? clusters * S : -1;
     return cache[dev][si];
@@ -350,33 +468,38 @@ inline int gemm_resident(int dev, int S, size_t smem) {
 
 // Split-K factor: the largest S in {1, 2, 4, 8} such that the S-CTA clusters
 // of all output tiles are resident at once, S divides the accumulator's
-// 4 x ceil(BN / 32) units and every rank keeps at least one K-step.
-template <int BN>
+// 4 x ceil(BN / 32) units and every rank keeps at least one K-range unit
+// (a K-step of 64 trits; 1.6-bit: a packed block of 320 trits).
+template <int FMT, int BN>
 inline int gemm_split(int dev, int M, int N, int K, size_t smem) {
     const int64_t tiles = (int64_t)((N + kGemmRows - 1) / kGemmRows) * ((M + BN - 1) / BN);
     const int units = 4 * ((BN + 31) / 32);
-    const int nk = (K + kGemmKStep - 1) / kGemmKStep;
+    const int ku = GemmSmem<FMT>::ksteps_per_w * kGemmKStep;
+    const int nk = (K + ku - 1) / ku;
     int S = 1;
     while (2 * S <= 8 && units % (2 * S) == 0 && 2 * S <= nk) {
-        const int r = gemm_resident<BN>(dev, 2 * S, smem);
+        const int r = gemm_resident<FMT, BN>(dev, 2 * S, smem);
         if (r <= 0 || tiles * 2 * S > r) break;
         S *= 2;
     }
     return S;
 }
 
-template <int BN>
+template <int FMT, int BN>
 inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
                           int64_t ldx, uint16_t *dY, int64_t ldy, int M, int N, int K,
                           cudaStream_t stream, int *last_cuda_error) {
+    using L = GemmSmem<FMT>;
     auto encode = tensor_map_encoder();
     if (!encode) return 5;  // TL_ERR_CUDA
     CUtensorMap tw, tx;
-    const int64_t rowbytes = ((int64_t)K + 3) / 4;
+    // packed row bytes: ceil(K / 4) (2-bit) or ceil(K / 5) (1.6-bit); boxes
+    // past the row's end read zeros, whose trits meet zero-filled activations
+    const int64_t rowbytes = FMT == 2 ? ((int64_t)K + 3) / 4 : ((int64_t)K + 4) / 5;
     {
         cuuint64_t dims[2] = {(cuuint64_t)rowbytes, (cuuint64_t)N};
         cuuint64_t strides[1] = {(cuuint64_t)ldp};
-        cuuint32_t box[2] = {16, kGemmRows};
+        cuuint32_t box[2] = {L::w_row_bytes, kGemmRows};
         cuuint32_t estr[2] = {1, 1};
         if (encode(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(dT), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -395,7 +518,7 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return 5;
     }
-    const size_t smem = gemm_smem_bytes(BN);
+    const size_t smem = gemm_smem_bytes<FMT>(BN);
     // the dynamic shared memory limit is a per-device function attribute
     constexpr int kMaxDev = 64;
     static std::once_flag attr_once[kMaxDev];
@@ -407,14 +530,14 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
         return 5;
     }
     std::call_once(attr_once[dev], [smem, dev] {
-        attr_err[dev] = cudaFuncSetAttribute(gemm2_kernel<BN>,
+        attr_err[dev] = cudaFuncSetAttribute(gemm_kernel<FMT, BN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     });
     if (attr_err[dev] != cudaSuccess) {
         *last_cuda_error = (int)attr_err[dev];
         return 5;
     }
-    const int S = gemm_split<BN>(dev, M, N, K, smem);
+    const int S = gemm_split<FMT, BN>(dev, M, N, K, smem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((N + kGemmRows - 1) / kGemmRows), (unsigned)((M + BN - 1) / BN),
                        (unsigned)S);
@@ -428,7 +551,7 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
     at[0].val.clusterDim.z = (unsigned)S;
     cfg.attrs = at;
     cfg.numAttrs = S > 1 ? 1 : 0;  // S = 1: a plain launch
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm2_kernel<BN>, tw, tx, alpha, dY, ldy, M, N, K);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN>, tw, tx, alpha, dY, ldy, M, N, K);
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;
@@ -437,15 +560,23 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
     return 0;
 }
 
+template <int FMT>
+inline int launch_gemm_fmt(const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
+                           int64_t ldx, uint16_t *dY, int64_t ldy, int M, int N, int K,
+                           cudaStream_t stream, int *err) {
+    if (M >= 256) return launch_gemm_bn<FMT, 256>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, err);
+    if (M >= 128) return launch_gemm_bn<FMT, 128>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, err);
+    if (M >= 64) return launch_gemm_bn<FMT, 64>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, err);
+    if (M >= 32) return launch_gemm_bn<FMT, 32>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, err);
+    return launch_gemm_bn<FMT, 16>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, err);
+}
+
 inline int launch_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
                        int64_t ldx, uint16_t *dY, int64_t ldy, int M, int N, int K,
                        cudaStream_t stream, int *last_cuda_error) {
-    if (fmt != 2) return 7;  // TL_ERR_UNSUPPORTED: the 1.6-bit tensor-core kernel is not built yet
-    if (M >= 256) return launch_gemm_bn<256>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
-    if (M >= 128) return launch_gemm_bn<128>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
-    if (M >= 64) return launch_gemm_bn<64>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
-    if (M >= 32) return launch_gemm_bn<32>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
-    return launch_gemm_bn<16>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
+    if (fmt == 2)
+        return launch_gemm_fmt<2>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
+    return launch_gemm_fmt<16>(dT, ldp, alpha, dX, ldx, dY, ldy, M, N, K, stream, last_cuda_error);
 }
 
 }  // namespace tlk
