@@ -477,6 +477,39 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     return out
 
 
+def time_ternarise(dev, stream, pk):
+    """Device ternariser on the largest sweep shapes: fp16 W read twice (the
+    exact |W| sum, then quantise + pack) and the packed rows written once."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    res = {}
+    for fmt in (2, 16):
+        for (N, K) in ((14336, 4096), (4096, 14336)):
+            g = torch.Generator(device=dev).manual_seed(N + K)
+            W = (torch.randn((N, K), generator=g, device=dev) * 0.02).half()
+            P = torch.empty((N, tl.padded_ldp(fmt, K)), dtype=torch.uint8, device=dev)
+            alpha = torch.empty(1, dtype=torch.float32, device=dev)
+            ws = torch.empty(tl.TERNARISE_WORKSPACE_BYTES, dtype=torch.uint8, device=dev)
+            with torch.cuda.stream(stream):
+                for _ in range(3):
+                    tl.ternarise(fmt, W, out=P, alpha=alpha, workspace=ws, stream=stream)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                reps = 10
+                a.record(stream)
+                for _ in range(reps):
+                    tl.ternarise(fmt, W, out=P, alpha=alpha, workspace=ws, stream=stream)
+                b.record(stream)
+                torch.cuda.synchronize()
+            us = a.elapsed_time(b) * 1e3 / reps
+            moved = 2 * (2 * N * K) + N * tl.row_bytes(fmt, K)
+            gbs = moved / (us * 1e-6) / 1e9
+            res[f"fmt{fmt}_N{N}_K{K}"] = {"us": round(us, 2), "GB/s": round(gbs, 1),
+                                         "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                                         "bytes": moved}
+            del W, P
+    return res
+
+
 def secondary(dev, stream, quick: bool):
     """1.6-bit sweep (p0 = 1/3), batched GEMM and the 30-layer decode step."""
     import torch
@@ -527,6 +560,10 @@ def secondary(dev, stream, quick: bool):
             del dP
         out[key] = gemm
     out["decode_step_30_layers"] = decode_step(dev, stream)
+    try:  # a failure here must not cost the lines above
+        out["ternarise"] = time_ternarise(dev, stream, pk)
+    except Exception as e:  # noqa: BLE001
+        out["ternarise"] = {"error": f"{type(e).__name__}: {e}"}
     # the same 2-bit sweep as twelve tl_gemv_ex calls per step (with and without PDL)
     sw = Sweep(2, dev)
     for flags, key in ((1, "gemv_2bit_sweep_per_call_pdl"), (0, "gemv_2bit_sweep_per_call")):

@@ -232,6 +232,34 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
 int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t *dX,
             int64_t ldx, uint16_t *dY, int64_t ldy, int M, int64_t N, int64_t K, void *stream);
 
+/* Device ternariser + packer: fp16 weights W [N][ldw] -> the shared scale
+ * *dAlpha and the packed trits P [N][ldp] (format fmt), the step before the
+ * layer: its weights are {-1, 0, 1} times one shared floating-point scale,
+ * obtained by rounding to the nearest ternary value ("Pith review of
+ * Spectra 1.1", "What carries the argument", and the round-to-nearest
+ * quantisation named among its domain assumptions).  The pages give no
+ * scale formula; this library takes
+ *   alpha = mean |W| over all N K entries: the sum of |w| is exact (integer
+ *           multiples of 2^-24), then alpha = fp32_rn(fp64_rn(fp64_rn(S) /
+ *           (N K)) * 2^-24), independent of the summation order;
+ *   t     = +1 if w > alpha / 2, -1 if w < -alpha / 2, else 0 (the nearest
+ *           ternary value to w / alpha in fp32, ties to 0; all-zero W gives
+ *           alpha = 0 and T = 0);
+ * and packs T exactly as tl_pack2 / tl_pack16 do (pad trits 0, bytes from
+ * the row's end to ldp written as 0).  W must be finite (NaN / Inf give
+ * unspecified T and alpha, never a fault).
+ * Device pointers, caller-owned: dW (16-byte aligned, ldw >= K, ldw % 8 ==
+ * 0), dP (16-byte aligned, ldp >= tl_packed_row_bytes, ldp % 16 == 0; must
+ * not overlap dW), dAlpha (one float, 4-byte aligned), dWorkspace
+ * (TL_TERNARISE_WORKSPACE_BYTES, 16-byte aligned, contents need no
+ * clearing; calls sharing it must be ordered on one stream).  Three
+ * stream-ordered launches, asynchronous, no allocation, may be captured
+ * into a CUDA graph.  Errors: TL_ERR_INVALID_ARG (format, null pointer,
+ * sizes), TL_ERR_ALIGN, TL_ERR_CUDA. */
+#define TL_TERNARISE_WORKSPACE_BYTES 16384u
+int tl_ternarise(int fmt, const uint16_t *dW, int64_t ldw, int64_t N, int64_t K, uint8_t *dP,
+                 int64_t ldp, float *dAlpha, void *dWorkspace, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the current device's error
  * word, which kernels set when one of their bounded waits gives up instead
  * of spinning forever.  Returns TL_OK, TL_ERR_TIMEOUT, or TL_ERR_CUDA if

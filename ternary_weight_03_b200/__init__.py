@@ -65,6 +65,7 @@ SIGNATURES = {
     "tl_gemv_batch_run": (_i32, [ctypes.POINTER(Plan), ctypes.c_uint, _p]),
     "tl_gemv_batch_plan_static": (_i32, [_i32, _i32, ctypes.POINTER(Layer), ctypes.POINTER(Plan)]),
     "tl_device_status": (_i32, [_p]),
+    "tl_ternarise": (_i32, [_i32, _p, _i64, _i64, _i64, _p, _i64, _p, _p, _p]),
 }
 
 
@@ -255,6 +256,28 @@ def gemv_batch_run(plan: Plan, stream=None, flags: int = 0):
     """Run a planned batch in one launch (asynchronous, graph-capturable)."""
     _check("tl_gemv_batch_run", lib().tl_gemv_batch_run(ctypes.byref(plan), int(flags),
                                                           _stream_ptr(stream)))
+
+
+TERNARISE_WORKSPACE_BYTES = 16384
+
+
+def ternarise(fmt: int, W, out=None, alpha=None, workspace=None, stream=None):
+    """Ternarise and pack fp16 weights W [N, K] (CUDA, row stride a multiple of
+    8) on the device: returns (P uint8 [N, ldp], alpha float32 [1]) with
+    alpha = mean |W| and P the packed nearest trits of W / alpha."""
+    import torch
+    assert W.dtype == torch.float16 and W.dim() == 2 and W.stride(1) == 1
+    N, K = W.shape
+    if out is None:
+        out = torch.empty((N, padded_ldp(fmt, K)), dtype=torch.uint8, device=W.device)
+    if alpha is None:
+        alpha = torch.empty(1, dtype=torch.float32, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(TERNARISE_WORKSPACE_BYTES, dtype=torch.uint8, device=W.device)
+    _check("tl_ternarise", lib().tl_ternarise(fmt, W.data_ptr(), W.stride(0), N, K,
+                                              out.data_ptr(), out.stride(0), alpha.data_ptr(),
+                                              workspace.data_ptr(), _stream_ptr(stream)))
+    return out, alpha
 
 
 def device_status(stream=None) -> int:

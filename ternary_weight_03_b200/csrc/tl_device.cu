@@ -1,6 +1,6 @@
 // tl_device.cu -- device entry points of libternary: argument validation,
-// kernel selection and launch for tl_gemv / tl_gemm / tl_gemv_batch, and the
-// device error word behind tl_device_status.
+// kernel selection and launch for tl_gemv / tl_gemm / tl_gemv_batch /
+// tl_ternarise, and the device error word behind tl_device_status.
 #include <cstdint>
 #include <mutex>
 #include <vector>
@@ -12,6 +12,7 @@
 #include "tl_gemm.cuh"
 #include "tl_gemv3.cuh"
 #include "tl_gemvp.cuh"
+#include "tl_ternarise.cuh"
 
 namespace {
 
@@ -170,6 +171,21 @@ int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t
     if (rc != TL_OK) return rc;
     return tlk::launch_gemm(fmt, dT, ldp, alpha, dX, ldx, dY, ldy, M, (int)N, (int)K,
                             (cudaStream_t)stream, &t_last_cuda_error);
+}
+
+int tl_ternarise(int fmt, const uint16_t *dW, int64_t ldw, int64_t N, int64_t K, uint8_t *dP,
+                 int64_t ldp, float *dAlpha, void *dWorkspace, void *stream) {
+    if (fmt != TL_FMT_2BIT && fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
+    if (!dW || !dP || !dAlpha || !dWorkspace) return TL_ERR_INVALID_ARG;
+    if (N < 1 || K < 1 || N > INT32_MAX || K > INT32_MAX - 512) return TL_ERR_INVALID_ARG;
+    if (ldw < K || ldp < tl_packed_row_bytes(fmt, K)) return TL_ERR_INVALID_ARG;
+    if (!aligned16(dW) || !aligned16(dP) || !aligned16(dWorkspace) || ((uintptr_t)dAlpha & 3u))
+        return TL_ERR_ALIGN;
+    if (ldw % 8 != 0 || ldp % 16 != 0) return TL_ERR_ALIGN;
+    const DeviceInfo *dev = device_info();
+    if (!dev) return TL_ERR_CUDA;
+    return tlk::launch_ternarise(fmt, dW, ldw, (int)N, (int)K, dP, ldp, dAlpha, dWorkspace,
+                                 dev->num_sms, (cudaStream_t)stream, &t_last_cuda_error);
 }
 
 int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes) {

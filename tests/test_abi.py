@@ -156,3 +156,24 @@ def test_batch_plan_and_run_rules(L):
     good = tl.Plan(fmt=2, count=2, max_m=1, total_items=3, total_tiles=2, dWorkspace=A,
                    workspace_bytes=n)
     assert L.tl_gemv_batch_run(ctypes.byref(good), 8, None) == 1   # unknown flag
+
+
+def ternarise_rc(L, fmt=2, dW=A, ldw=1024, N=64, K=1024, dP=A, ldp=256, dAlpha=A, ws=A):
+    return L.tl_ternarise(fmt, dW, ldw, N, K, dP, ldp, dAlpha, ws, None)
+
+
+@pytest.mark.parametrize("kw,rc", [
+    (dict(fmt=4), 1), (dict(dW=0), 1), (dict(dP=0), 1), (dict(dAlpha=0), 1), (dict(ws=0), 1),
+    (dict(N=0), 1), (dict(K=0), 1), (dict(N=-1), 1), (dict(N=2 ** 31), 1),
+    (dict(ldw=1016), 1), (dict(ldp=240), 1), (dict(fmt=16, ldp=192), 1),
+    (dict(dW=A + 8), 4), (dict(dP=A + 4), 4), (dict(ws=A + 8), 4), (dict(dAlpha=A + 2), 4),
+    (dict(ldw=1028), 4), (dict(ldp=264), 4),
+])
+def test_ternarise_argument_rules(L, kw, rc):
+    assert ternarise_rc(L, **kw) == rc
+
+
+def test_ternarise_workspace_constant():
+    text = HEADER.read_text()
+    m = re.search(r"#define TL_TERNARISE_WORKSPACE_BYTES (\d+)u", text)
+    assert m and int(m.group(1)) == tl.TERNARISE_WORKSPACE_BYTES
