@@ -653,7 +653,10 @@ def run_gpu(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if not args.no_secondary:
-        line["secondary"] = secondary(dev, stream, quick=True)
+        try:  # context lines: an error there is recorded, the headline line still prints
+            line["secondary"] = secondary(dev, stream, quick=True)
+        except Exception as e:  # noqa: BLE001
+            line["secondary"] = {"error": f"{type(e).__name__}: {e}"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
