@@ -555,8 +555,13 @@ def secondary(dev, stream, quick: bool):
                     torch.cuda.synchronize()
                 us = a.elapsed_time(b) * 1e3 / reps
                 tf = 2.0 * M * N * K / (us * 1e-6) / 1e12
+                # small M is bound by HBM: packed weights + X + Y once
+                moved = N * tl.row_bytes(fmt, K) + 2 * M * K + 2 * M * N
+                gbs = moved / (us * 1e-6) / 1e9
                 gemm[f"M{M}_K{K}_N{N}"] = {"us": round(us, 2), "TFLOP/s": round(tf, 1),
-                                           "frac_tensor": round(tf / pk["bf16_tflops"], 4)}
+                                           "frac_tensor": round(tf / pk["bf16_tflops"], 4),
+                                           "GB/s": round(gbs, 1),
+                                           "frac_hbm": round(gbs / pk["hbm_gbs"], 4)}
             del dP
         out[key] = gemm
     out["decode_step_30_layers"] = decode_step(dev, stream)

@@ -249,8 +249,9 @@ int tl_gemm(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint16_t
  * the row's end to ldp written as 0).  W must be finite (NaN / Inf give
  * unspecified T and alpha, never a fault).
  * Device pointers, caller-owned: dW (16-byte aligned, ldw >= K, ldw % 8 ==
- * 0), dP (16-byte aligned, ldp >= tl_packed_row_bytes, ldp % 16 == 0; must
- * not overlap dW), dAlpha (one float, 4-byte aligned), dWorkspace
+ * 0), dP (16-byte aligned, tl_packed_row_bytes <= ldp <= INT32_MAX,
+ * ldp % 16 == 0; must not overlap dW), dAlpha (one float, 4-byte aligned),
+ * dWorkspace
  * (TL_TERNARISE_WORKSPACE_BYTES, 16-byte aligned, contents need no
  * clearing; calls sharing it must be ordered on one stream).  Three
  * stream-ordered launches, asynchronous, no allocation, may be captured

@@ -178,7 +178,7 @@ int tl_ternarise(int fmt, const uint16_t *dW, int64_t ldw, int64_t N, int64_t K,
     if (fmt != TL_FMT_2BIT && fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
     if (!dW || !dP || !dAlpha || !dWorkspace) return TL_ERR_INVALID_ARG;
     if (N < 1 || K < 1 || N > INT32_MAX || K > INT32_MAX - 512) return TL_ERR_INVALID_ARG;
-    if (ldw < K || ldp < tl_packed_row_bytes(fmt, K)) return TL_ERR_INVALID_ARG;
+    if (ldw < K || ldp < tl_packed_row_bytes(fmt, K) || ldp > INT32_MAX) return TL_ERR_INVALID_ARG;
     if (!aligned16(dW) || !aligned16(dP) || !aligned16(dWorkspace) || ((uintptr_t)dAlpha & 3u))
         return TL_ERR_ALIGN;
     if (ldw % 8 != 0 || ldp % 16 != 0) return TL_ERR_ALIGN;

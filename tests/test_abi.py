@@ -165,7 +165,7 @@ def ternarise_rc(L, fmt=2, dW=A, ldw=1024, N=64, K=1024, dP=A, ldp=256, dAlpha=A
 @pytest.mark.parametrize("kw,rc", [
     (dict(fmt=4), 1), (dict(dW=0), 1), (dict(dP=0), 1), (dict(dAlpha=0), 1), (dict(ws=0), 1),
     (dict(N=0), 1), (dict(K=0), 1), (dict(N=-1), 1), (dict(N=2 ** 31), 1),
-    (dict(ldw=1016), 1), (dict(ldp=240), 1), (dict(fmt=16, ldp=192), 1),
+    (dict(ldw=1016), 1), (dict(ldp=240), 1), (dict(fmt=16, ldp=192), 1), (dict(ldp=2 ** 32), 1),
     (dict(dW=A + 8), 4), (dict(dP=A + 4), 4), (dict(ws=A + 8), 4), (dict(dAlpha=A + 2), 4),
     (dict(ldw=1028), 4), (dict(ldp=264), 4),
 ])
