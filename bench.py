@@ -477,6 +477,40 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     return out
 
 
+def time_single_cold(dev, stream, pk):
+    """K = N = 1024, M = 1, 2-bit, alpha = 0.02 (262,144 packed bytes): one
+    tl_gemv_ex call at a time, L2 flushed by a 256 MiB write before each,
+    median of 20 calls.  Latency-bound: the figure is the call's latency."""
+    import numpy as np
+    import torch
+    import synth
+    import ternary_weight_03_b200 as tl
+    P, _, _ = make_matrix(2, 1024, 1024, 0)
+    dP = torch.from_numpy(P).to(dev)
+    X = torch.from_numpy(synth.activations(0, 1, 1024)).to(dev)
+    Y = torch.empty((1, 1024), dtype=torch.float16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(23):
+            flush.fill_(i & 255)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            rc = tl.lib().tl_gemv_ex(2, dP.data_ptr(), dP.stride(0), 0.02, X.data_ptr(), 1024,
+                                     Y.data_ptr(), 1024, 1, 1024, 1024, 0, stream.cuda_stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            if rc != 0:
+                return {"status": tl.status_str(rc)}
+            if i >= 3:
+                times.append(a.elapsed_time(b) * 1e3)
+    us = float(np.median(times))
+    gbs = 1024 * 256 / (us * 1e-6) / 1e9
+    return {"us_median": round(us, 2), "GB/s": round(gbs, 1),
+            "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "l2": "flushed by a 256 MiB write before every call"}
+
+
 def time_ternarise(dev, stream, pk):
     """Device ternariser on the largest sweep shapes: fp16 W read twice (the
     exact |W| sum, then quantise + pack) and the packed rows written once."""
@@ -511,7 +545,9 @@ def time_ternarise(dev, stream, pk):
 
 
 def secondary(dev, stream, quick: bool):
-    """1.6-bit sweep (p0 = 1/3), batched GEMM and the 30-layer decode step."""
+    """1.6-bit sweep (p0 = 1/3), batched GEMM (both formats), the 30-layer
+    decode step, the device ternariser, the cold 1024 x 1024 single call and
+    the sweep as separate per-layer calls."""
     import torch
     import ternary_weight_03_b200 as tl
     out = {}
@@ -565,10 +601,12 @@ def secondary(dev, stream, quick: bool):
             del dP
         out[key] = gemm
     out["decode_step_30_layers"] = decode_step(dev, stream)
-    try:  # a failure here must not cost the lines above
-        out["ternarise"] = time_ternarise(dev, stream, pk)
-    except Exception as e:  # noqa: BLE001
-        out["ternarise"] = {"error": f"{type(e).__name__}: {e}"}
+    for key, fn in (("ternarise", time_ternarise),
+                    ("gemv_2bit_1024x1024_m1_cold", time_single_cold)):
+        try:  # a failure here must not cost the other lines
+            out[key] = fn(dev, stream, pk)
+        except Exception as e:  # noqa: BLE001
+            out[key] = {"error": f"{type(e).__name__}: {e}"}
     # the same 2-bit sweep as twelve tl_gemv_ex calls per step (with and without PDL)
     sw = Sweep(2, dev)
     for flags, key in ((1, "gemv_2bit_sweep_per_call_pdl"), (0, "gemv_2bit_sweep_per_call")):
