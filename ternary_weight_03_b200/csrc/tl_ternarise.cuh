@@ -91,8 +91,10 @@ absum_kernel(const uint16_t *__restrict__ W, int64_t ldw, int N, int K, U128 *pa
         const int k0 = 16 * u;
         uint64_t s = 0;  // 16 x < 2^41
         if (k0 + 16 <= K) {
-            const uint4 a = __ldcs(reinterpret_cast<const uint4 *>(row + k0));
-            const uint4 b = __ldcs(reinterpret_cast<const uint4 *>(row + k0) + 1);
+            // cached loads: pass 3 reads W again, and a matrix below the L2's
+            // size can partly stay there; pass 3 streams it out (last use)
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(row + k0));
+            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(row + k0) + 1);
             const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i)
