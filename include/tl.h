@@ -59,7 +59,7 @@ enum tl_status {
     TL_ERR_ALIGN = 4,       /* a device pointer or stride breaks the alignment rules */
     TL_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed */
     TL_ERR_TIMEOUT = 6,     /* a kernel's bounded wait ran out (see tl_device_status) */
-    TL_ERR_UNSUPPORTED = 7  /* no kernel for this (format, shape) on this device */
+    TL_ERR_UNSUPPORTED = 7  /* reserved: no kernel for a (format, shape); no call returns it now */
 };
 
 /* Static, human-readable name of a status code (never NULL). */
