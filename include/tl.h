@@ -155,14 +155,24 @@ typedef struct tl_gemv_layer {
  * Plain data owned by the caller; treat the fields as read-only. */
 typedef struct tl_gemv_plan {
     int fmt, count, max_m, total_items, total_tiles;
+    int total_units;  /* activation conversion units of the launch */
+    int chained;      /* 1 if some layer has TL_LAYER_READS_EARLIER */
     void *dWorkspace;
     size_t workspace_bytes;
+    uint64_t generation; /* 0, or the static plan's number (tl_gemv_batch_plan_static) */
 } tl_gemv_plan;
 
-/* Workspace bytes a batch needs: the layer table and one TMA descriptor per
- * layer (~200 B per layer), counters, and fp32 partial sums of the layers
- * whose rows are split across CTAs (about N * M * 4 * K / 2048 bytes per
- * such layer).  Validates the batch like tl_gemv_batch_plan.  Pure host
+/* Workspace bytes a batch needs.  2-bit: counters, one TMA descriptor per
+ * layer, a 96-byte record per work item (128 output rows x about 4096 trits
+ * of K), the layers' activations converted once into the tensor-core operand
+ * layout (per 1024 trits of K: 8 KB at M = 1, 16 KB at M = 2, 2 KB per token
+ * rounded up to even at M >= 3, plus 64 B; none for TL_LAYER_READS_EARLIER
+ * layers, which convert on chip) with a 48-byte record per 1024 trits and
+ * token, and 8-byte partial sums of rows split into K-parts (N * M * 8 bytes
+ * per part).  1.6-bit: the layer table and one TMA descriptor per layer
+ * (~200 B per layer), counters, and fp32 partial sums of the layers whose
+ * rows are split across CTAs (about N * M * 4 * K / 2048 bytes per such
+ * layer).  Validates the batch like tl_gemv_batch_plan.  Pure host
  * function. */
 int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes);
 
@@ -195,10 +205,13 @@ int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dW
  * TL_STATIC_WORKSPACE_BYTES is rejected with TL_ERR_INVALID_ARG before
  * anything is written.  Races: the array is shared by every caller in the
  * process on that device, so planning again replaces the previous static
- * plan (a plan filled earlier then runs on the new table); keep one static
- * plan per device in use at a time and do not plan from several host
- * threads at once.  The call synchronizes the device first, so no run of an
- * earlier static plan is still reading the array when it is rewritten.
+ * plan.  Each static plan carries a per-device number (plan->generation);
+ * the call takes a new number before it writes the array, and
+ * tl_gemv_batch_run returns TL_ERR_INVALID_ARG, without launching, for a
+ * static plan whose number is no longer the device's latest (or that was
+ * planned on another device): plan again instead.  Do not plan from several
+ * host threads at once.  The call synchronizes the device first, so no run
+ * of an earlier static plan is still reading the array when it is rewritten.
  * Clearing: the call zeroes the array's counters; every completed
  * tl_gemv_batch_run leaves them zero; after a run that ends in
  * TL_ERR_TIMEOUT, plan again before the next run.  Otherwise as
@@ -218,8 +231,9 @@ int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
  * the first weights are fetched while the preceding kernel finishes; X, Y
  * and the workspace counters are touched only after it completed).
  * Asynchronous, allocates nothing, may be captured into a CUDA graph.
- * Errors: TL_ERR_INVALID_ARG (plan not filled by tl_gemv_batch_plan, bad
- * flags), TL_ERR_CUDA. */
+ * Errors: TL_ERR_INVALID_ARG (plan not filled by tl_gemv_batch_plan, a
+ * static plan replaced by a later tl_gemv_batch_plan_static, bad flags),
+ * TL_ERR_CUDA. */
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream);
 
 /* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and

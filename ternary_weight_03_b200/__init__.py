@@ -42,7 +42,9 @@ class Plan(ctypes.Structure):
     """tl_gemv_plan: a planned batch (filled by tl_gemv_batch_plan)."""
     _fields_ = [("fmt", ctypes.c_int), ("count", ctypes.c_int), ("max_m", ctypes.c_int),
                 ("total_items", ctypes.c_int), ("total_tiles", ctypes.c_int),
-                ("dWorkspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t)]
+                ("total_units", ctypes.c_int), ("chained", ctypes.c_int),
+                ("dWorkspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+                ("generation", ctypes.c_uint64)]
 
 
 # (name, restype, argtypes) of every symbol the C header declares

@@ -1,0 +1,1299 @@
+// tl_decode.cuh -- a batch of decode-shaped 2-bit ternary layers (M = 1..8
+// tokens each) in ONE persistent launch:
+//   for every layer l:  Y_l[m][n] = fp16_rn(alpha_l * sum_k T_l[n][k] X_l[m][k]).
+//
+// Decoding streams every packed weight once and is bound by memory bandwidth
+// ("Pith review of Spectra 1.1", "What carries the argument"), so the kernel
+// is built around keeping HBM busy: one CTA per SM walks a queue of work
+// items (layer, 128-row tile, K-part) across all layers of the batch, and the
+// instructions spent per packed byte must stay far below what the SM can
+// issue.  Two tensor-core engines, chosen per item by its token count:
+//
+//  * M <= 2, exact integer engine (mma.sync m16n8k32, u8 x u8 -> s32).  A
+//    holds the 2-bit digits d = t + 1 of one digit position j of every byte
+//    of a packed word, left in place (one AND: values d * 4^j), with one
+//    accumulator per position.  B holds the activations as exact integers:
+//    every binary16 x has x * 2^24 integral and |x * 2^24| < 2^40, so
+//    z = x * 2^24 + 2^40 is a 41-bit natural number, stored as six u8 planes
+//    (B columns), next to one column of ones.  Then
+//      sum_k t_k x_k * 2^24 = sum_p 256^p S_p - 2^40 S_1 - Q,
+//    with S_p = sum_k d_k u_p(k) (MMA columns, exact in s32 per item),
+//    S_1 = sum_k d_k (the ones column) and Q = sum_k x_k 2^24 (exact).  The
+//    sum is exact in int64, so a layer's result is the single rounding
+//    fp16_rn(alpha * V * 2^-24) whatever the split of K.
+//  * M >= 3, fp16 engine (mma.sync m16n8k16, fp16 -> fp32): masking digit
+//    position j of every byte of a packed word leaves the digits as subnormal
+//    halves d * 2^(2j-24) (one AND per register); one accumulator per digit
+//    position, combined with exact power-of-two scales; sum_k x_k is
+//    subtracted at the end (d = t + 1).
+//
+// Weights arrive by TMA in 128-byte-wide boxes of 128 rows with the 128-byte
+// swizzle, two boxes per stage (256 packed bytes = 1024 trits per row).  A
+// consumer lane (g, c) reads 16-byte chunk 4v + c of rows g and g + 8 of a
+// 16-row tile; MMA row g is physical row pi(g) = ((g & 1) << 2) | (g >> 1), so
+// the two rows of every quarter-warp differ in bit 2 and each LDS.128 touches
+// every bank once.
+//
+// Activations go into the B layout of their engine once per (layer, stage),
+// not once per item: every warp except the producer first converts such
+// units (handed out through a workspace counter) into the workspace and
+// counts them per layer; a stage's converted operands then arrive by one
+// bulk copy next to its weights.  Layers flagged as reading an earlier
+// layer's output (their X is written during this launch) are converted per
+// item instead, from raw activations, by stager warps.
+//
+// Warp roles of a CTA (704 threads):
+//  * warp 0, producer: issues each stage's copies into a ring and queues items
+//    (items come from a workspace counter, fetched one item ahead);
+//  * warps 1..3, stagers (warp 1 + i owns the ring slots s with s mod 3 = i);
+//  * warps 4, 5, epilogues (alternate items): sum the consumer partials of an
+//    item in a fixed order, then write Y, or a partial of a split tile to the
+//    workspace where the last part to arrive adds the parts in part order;
+//  * warps 6..21, consumers: warp w takes row tiles 2 (w & 3) and 2 (w & 3) + 1
+//    and the quarter w >> 2 of every stage (segment (w >> 3), chunks
+//    4 ((w >> 2) & 1) .. +3).
+// The cross-warp and cross-CTA sums follow the pages' shared-memory tree
+// reduction of per-warp partials (Figure 11 caption text on appendix G.4 of the
+// same page), in a fixed order.  All waits are bounded; a timeout sets the
+// device error word.  The last CTA to finish resets the workspace counters, so
+// they stay zero between launches.
+#pragma once
+#include <cuda.h>
+#include <cstring>
+#include <mutex>
+#include <vector>
+#include "tl_common.cuh"
+#include "tl_sm100.cuh"
+
+namespace tlk {
+
+constexpr int kDkTiles = 8;                              // 16-row MMA tiles per item
+constexpr int kDkRows = 16 * kDkTiles;                   // 128 weight rows per item
+constexpr int kDkSegBytes = 128;                         // packed bytes per row per TMA box
+constexpr int kDkStageW = 2 * kDkSegBytes;               // packed bytes per row per stage
+constexpr int kDkStageTrits = 4 * kDkStageW;             // 1024 activations per stage
+constexpr int kDkBoxBytes = kDkRows * kDkSegBytes;       // 16 KB
+constexpr int kDkWBytes = 2 * kDkBoxBytes;               // 32 KB of weights per stage
+constexpr int kDkRawTok = 2 * kDkStageTrits;             // 2 KB of fp16 activations per token
+constexpr int kDkConsumers = 16;
+constexpr int kDkStagers = 3;
+constexpr int kDkEpilogues = 2;
+constexpr int kDkFirstEpi = 1 + kDkStagers;
+constexpr int kDkFirstCons = kDkFirstEpi + kDkEpilogues;
+constexpr int kDkWarps = kDkFirstCons + kDkConsumers;  // 22
+constexpr int kDkThreads = 32 * kDkWarps;              // 704
+constexpr int kDkMaxStages = 6;
+constexpr int kDkQueue = 16;
+constexpr int kDkPartBufs = 2;
+constexpr int kDkImmaMaxM = 2;                          // exact integer engine up to 2 tokens
+constexpr int kDkItemStages = 4;                        // target stages per item
+constexpr int kDkMaxItemStages = 32;                    // s32 sums of an item stay exact
+constexpr uint32_t kDkSmemBudget = 232448u;             // 227 KB
+constexpr int kDkMetaBytes = 64;                        // per stage: per-token offsets, first
+
+// Workspace counters (u32 words of the 256-byte header).
+constexpr int kDkCtrFinal = 1;      // tiles whose outputs are stored
+constexpr int kDkCtrDone = 2;       // CTAs that have finished
+constexpr int kDkCtrItems = 3;      // items handed out beyond the first gridDim.x
+constexpr int kDkCtrUnits = 4;      // conversion units handed out
+constexpr int kDkCtrUnitsDone = 5;  // conversion units written
+
+// Bytes of converted B operands of one stage of a layer with M tokens: the
+// integer engine needs 8 KB per column group (2 groups at M = 2), the fp16
+// engine 1 KB per token and segment (tokens rounded up to even).
+__host__ __device__ constexpr uint32_t dk_stage_b(int M) {
+    return M <= 1 ? 8192u : (M == 2 ? 16384u : 2048u * (uint32_t)(M + (M & 1)));
+}
+// Consumer -> epilogue buffer: [token][warp][tile][row] of int64 (M <= 2) or fp32.
+__host__ __device__ constexpr uint32_t dk_part_bytes(int maxM) {
+    return (maxM <= 1 ? 4096u : 8192u) > 2048u * (uint32_t)maxM ? (maxM <= 1 ? 4096u : 8192u)
+                                                                 : 2048u * (uint32_t)maxM;
+}
+
+// One work item as the producer reads it (96 bytes): everything the CTA's
+// roles need, so no lookup chain stands between items.
+struct DkItemRec {
+    const uint16_t *X;
+    uint16_t *Y;
+    const uint8_t *B;  // converted operands of the layer ([meta][B] per stage), or null
+    int64_t part_off;  // first 8-byte partial slot of the item's layer
+    float alpha;
+    int layer;         // index of the layer's tensor map
+    int tile, part, s0, s1;
+    int M, K, N, ldx, ldy;
+    int parts;         // K-parts per tile of the layer
+    int tile_begin;    // global index of the layer's first tile
+    int wait_tiles;    // tiles that must be final before X is read (0: none)
+    int need;          // conversion units of the layer (stages x M)
+    int bstride;       // bytes per stage of B (64 + dk_stage_b(M))
+};
+static_assert(sizeof(DkItemRec) == 96, "item record is six 16-byte loads");
+
+// One conversion unit: one stage of one token of one layer.
+struct DkUnitRec {
+    const uint16_t *X;  // the layer's activations
+    uint8_t *dst;       // [meta][B] of (layer, stage)
+    int layer, stage, m, M, K, ldx;
+    int pad_[2];
+};
+static_assert(sizeof(DkUnitRec) == 48, "unit record is three 16-byte loads");
+
+// Workspace layout (every region 256-byte aligned):
+//   header  : 64 u32 counters (kDkCtr*)
+//   maps    : count x CUtensorMap
+//   items   : total_items x DkItemRec
+//   units   : total_units x DkUnitRec
+//   ready   : count x u32, conversion units written per layer
+//   tiles   : total_tiles x u32, parts of each tile that have arrived
+//   partials: 8-byte partial sums of split tiles (int64 for M <= 2, double above)
+//   staged  : converted operands, per layer stages x (64 + dk_stage_b(M)) bytes
+struct DkWsLayout {
+    size_t maps, items, units, ready, tiles, partials, staged, total;
+    DkWsLayout(int count, int total_items, int total_units, int total_tiles, int64_t slots,
+               int64_t staged_bytes) {
+        auto up = [](size_t v) { return (v + 255u) & ~(size_t)255u; };
+        maps = 256;
+        items = up(maps + (size_t)count * sizeof(CUtensorMap));
+        units = up(items + (size_t)total_items * sizeof(DkItemRec));
+        ready = up(units + (size_t)total_units * sizeof(DkUnitRec));
+        tiles = up(ready + (size_t)count * 4u);
+        partials = up(tiles + (size_t)total_tiles * 4u);
+        staged = up(partials + (size_t)slots * 8u);
+        total = up(staged + (size_t)staged_bytes);
+    }
+};
+
+struct DkArgs {
+    uint32_t *ctr;
+    const CUtensorMap *maps;
+    const DkItemRec *items;
+    const DkUnitRec *units;
+    uint32_t *ready;
+    uint32_t *tile_ctr;
+    int64_t *partials;
+    int count;
+    int total_items;
+    int total_units;
+    int maxM;
+    int chained;  // some layer converts per item (raw activation buffers needed)
+};
+
+struct DkQEntry {
+    uint16_t *Y;
+    int64_t part_off;
+    float alpha;
+    int item;  // -1: no more items
+    int tile, part, s0, s1, M, K, N, ldy, parts, tile_begin, pre;
+    int pad_;
+};
+
+struct DkLayout {
+    uint32_t ns, raw_stage, slot_b, parts, w_off, raw_off, st_off, part_off, q_off, bar_off, total;
+    __host__ __device__ DkLayout(int maxM, int chained) {
+        raw_stage = chained ? (uint32_t)kDkRawTok * (uint32_t)maxM : 0u;
+        slot_b = (maxM <= 1 ? 8192u : 16384u) + kDkMetaBytes;  // [meta][B]
+        parts = dk_part_bytes(maxM);
+        const uint32_t per_stage = (uint32_t)kDkWBytes + raw_stage + slot_b;
+        const uint32_t fixed = kDkPartBufs * parts + kDkQueue * (uint32_t)sizeof(DkQEntry) +
+                               8u * (3u * kDkMaxStages + 2u * kDkQueue + 2u * kDkPartBufs) +
+                               1024u;  // alignment slack of the dynamic base
+        const uint32_t n = (kDkSmemBudget - fixed) / per_stage;
+        ns = n > (uint32_t)kDkMaxStages ? (uint32_t)kDkMaxStages : n;  // >= 3 for maxM <= 8
+        w_off = 0;
+        raw_off = ns * (uint32_t)kDkWBytes;
+        st_off = raw_off + ns * raw_stage;
+        part_off = st_off + ns * slot_b;
+        q_off = part_off + kDkPartBufs * parts;
+        bar_off = (q_off + kDkQueue * (uint32_t)sizeof(DkQEntry) + 7u) & ~7u;
+        total = bar_off + 8u * (3u * ns + 2u * kDkQueue + 2u * kDkPartBufs) + 1024u;
+    }
+};
+
+template <typename R, int N16>
+__device__ __forceinline__ R dk_load_rec(const R *base, int idx) {
+    const uint4 *p = reinterpret_cast<const uint4 *>(base + idx);
+    uint4 v[N16];
+#pragma unroll
+    for (int i = 0; i < N16; ++i) v[i] = __ldg(p + i);
+    R r;
+    memcpy(&r, v, sizeof(r));
+    return r;
+}
+
+__device__ __forceinline__ void dk_bulk_load(void *smem_dst, const void *src, uint32_t bytes,
+                                             uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void dk_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ uint32_t dk_ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+// Orders this thread's generic-proxy accesses to global memory with its
+// async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void dk_fence_proxy_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ bool dk_warp_wait(uint64_t *bar, uint32_t parity) {
+    const bool ok = mbar_wait(bar, parity);
+    return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool dk_next_item(const DkQEntry *queue, uint64_t *qfull,
+                                             uint64_t *qempty, int &qi, DkQEntry &e) {
+    const int q = qi % kDkQueue;
+    if (!dk_warp_wait(&qfull[q], (uint32_t)(qi / kDkQueue) & 1u)) return false;
+    e = queue[q];
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&qempty[q]);
+    ++qi;
+    return e.item >= 0;
+}
+// Lane 0 spins (bounded) until *p >= target, or until *all_p >= all_target
+// when all_p is given (then *all_seen is set); false on a timeout.  The
+// result is the same in every lane.
+__device__ __forceinline__ bool dk_wait_count(const uint32_t *p, uint32_t target,
+                                              const uint32_t *all_p, uint32_t all_target,
+                                              bool *all_seen) {
+    bool good = true, all = false;
+    if ((threadIdx.x & 31) == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (true) {
+            if (all_p && dk_ld_acquire(all_p) >= all_target) {
+                all = true;
+                break;
+            }
+            if (dk_ld_acquire(p) >= target) break;
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(&g_error_word, kErrTimeout);
+                good = false;
+                break;
+            }
+            __nanosleep(64);
+        }
+    }
+    all = __shfl_sync(0xffffffffu, all ? 1 : 0, 0) != 0;
+    if (all_seen && all) *all_seen = true;
+    return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+}
+
+__device__ __forceinline__ uint4 dk_lds128(const uint8_t *p) {
+    return *reinterpret_cast<const uint4 *>(p);
+}
+__device__ __forceinline__ uint32_t dk_word(const uint4 &v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// D (16x8 s32) += A (16x32 u8, row) * B (32x8 u8, col)
+__device__ __forceinline__ void mma_u8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Integer engine: B column of token m's plane p, and of the ones column.
+__host__ __device__ constexpr int dk_col(int m, int p) { return 6 * m + p; }
+__host__ __device__ constexpr int dk_ones_col(int M) { return 6 * M; }
+
+// Offset of the 16-byte B block of (16-trit word w of the stage, column col)
+// in the integer engine's layout: [cg][segment][v][i][col & 7][c], where
+// w = segment * 32 + (4 v + c) * 4 + i.  A consumer quarter-warp reads two
+// columns x four c: 128 contiguous bytes.
+__device__ __forceinline__ uint32_t dk_iblock(int w, int col) {
+    const int h = w >> 5, ch = (w >> 2) & 7, i = w & 3, v = ch >> 2, c = ch & 3;
+    return (uint32_t)((col >> 3) * 8192 + h * 4096 + (((v * 4 + i) * 8 + (col & 7)) * 4 + c) * 16);
+}
+// fp16 engine: offset of the 16-byte half `hf` (digit positions 2hf, 2hf+1)
+// of the B operands of (word w, token m): [segment][v][i][hf][m][c], Mp =
+// tokens rounded up to even (a quarter-warp reads tokens 2p, 2p+1 x four c).
+__device__ __forceinline__ uint32_t dk_hblock(int w, int m, int hf, int Mp) {
+    const int h = w >> 5, ch = (w >> 2) & 7, i = w & 3, v = ch >> 2, c = ch & 3;
+    return (uint32_t)(h * 1024 * Mp + ((((v * 4 + i) * 2 + hf) * Mp + m) * 4 + c) * 16);
+}
+
+// MMA row g of a 16-row tile reads physical row pi(g) (and pi(g) + 8).
+__host__ __device__ constexpr int dk_pi(int g) { return ((g & 1) << 2) | (g >> 1); }
+__host__ __device__ constexpr int dk_pi_inv(int p) { return ((p & 3) << 1) | (p >> 2); }
+
+// The 16 activations of word w (elements 16w .. 16w + 15 of a stage that
+// starts at src), zero at elements >= valid.  Only whole 8-element halves that
+// start below `valid` are read, so reads of global activations stay inside
+// the row (ldx is a multiple of 8 and >= K).
+__device__ __forceinline__ void dk_read_word(const uint16_t *src, int w, int valid,
+                                             uint32_t (&r)[8]) {
+    const int e0 = 16 * w;
+    uint4 lo = make_uint4(0u, 0u, 0u, 0u), hi = lo;
+    if (e0 < valid) lo = *reinterpret_cast<const uint4 *>(src + e0);
+    if (e0 + 8 < valid) hi = *reinterpret_cast<const uint4 *>(src + e0 + 8);
+    r[0] = lo.x; r[1] = lo.y; r[2] = lo.z; r[3] = lo.w;
+    r[4] = hi.x; r[5] = hi.y; r[6] = hi.z; r[7] = hi.w;
+    const int keep = valid - e0;
+    if (keep < 16) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t l = 2 * i < keep ? 0x0000FFFFu : 0u;
+            const uint32_t h = 2 * i + 1 < keep ? 0xFFFF0000u : 0u;
+            r[i] &= l | h;
+        }
+    }
+}
+
+// One warp converts one stage of token m for the integer engine: z = x 2^24 +
+// 2^40 as six u8 planes, each 16-byte block the 4x4 transpose of a word's
+// elements (byte 4j + b = element 4b + j), the ones column (m == 0), and
+// Q = sum x 2^24 into meta[m] (exact: the partial sums of binary16 values are
+// multiples of 2^-24 below 2^26, within a double's 53 bits).
+__device__ __forceinline__ void dk_conv_imma(const uint16_t *src, int valid, int m, int M,
+                                             uint8_t *dstB, uint8_t *meta, int lane) {
+    const int ones = dk_ones_col(M);
+    double qd = 0.0;
+    for (int w = lane; w < 64; w += 32) {
+        uint32_t r[8];
+        dk_read_word(src, w, valid, r);
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int e2 = 0; e2 < 16; e2 += 2) {
+            const float2 xf2 = __half22float2(*reinterpret_cast<const __half2 *>(&r[e2 >> 1]));
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float xf = u ? xf2.y : xf2.x;
+                const float fl = floorf(xf);
+                lo[e2 + u] = (uint32_t)((xf - fl) * 16777216.0f);
+                hi[e2 + u] = (uint32_t)(fl + 65536.0f);
+                qd += (double)xf;
+            }
+        }
+        // bytes 0..2 of lo[] are planes 0..2, bytes 0..2 of hi[] planes 3..5
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const uint32_t *s = half ? hi : lo;
+            uint32_t pl[3][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t A0 = prmt(s[j], s[4 + j], 0x5140u);
+                const uint32_t B0 = prmt(s[8 + j], s[12 + j], 0x5140u);
+                const uint32_t C0 = prmt(s[j], s[4 + j], 0x7362u);
+                const uint32_t D0 = prmt(s[8 + j], s[12 + j], 0x7362u);
+                pl[0][j] = prmt(A0, B0, 0x5410u);
+                pl[1][j] = prmt(A0, B0, 0x7632u);
+                pl[2][j] = prmt(C0, D0, 0x5410u);
+            }
+#pragma unroll
+            for (int p = 0; p < 3; ++p)
+                *reinterpret_cast<uint4 *>(dstB + dk_iblock(w, dk_col(m, 3 * half + p))) =
+                    make_uint4(pl[p][0], pl[p][1], pl[p][2], pl[p][3]);
+        }
+        if (m == 0)
+            *reinterpret_cast<uint4 *>(dstB + dk_iblock(w, ones)) =
+                make_uint4(0x01010101u, 0x01010101u, 0x01010101u, 0x01010101u);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, o);
+    if (lane == 0) reinterpret_cast<int64_t *>(meta)[m] = (int64_t)(qd * 16777216.0);
+}
+
+// One warp converts one stage of token m for the fp16 engine: per word and
+// digit position j the pairs (x_j, x_{8+j}) and (x_{4+j}, x_{12+j}), and
+// sum_k x into meta[m] (fp32).
+__device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, int valid, int m, int Mp,
+                                             uint8_t *dstB, uint8_t *meta, int lane) {
+    float sx = 0.f;
+    for (int w = lane; w < 64; w += 32) {
+        uint32_t r[8];
+        dk_read_word(src, w, valid, r);
+        uint32_t b[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
+            b[2 * j] = prmt(r[j >> 1], r[4 + (j >> 1)], sel);
+            b[2 * j + 1] = prmt(r[2 + (j >> 1)], r[6 + (j >> 1)], sel);
+        }
+        *reinterpret_cast<uint4 *>(dstB + dk_hblock(w, m, 0, Mp)) = make_uint4(b[0], b[1], b[2], b[3]);
+        *reinterpret_cast<uint4 *>(dstB + dk_hblock(w, m, 1, Mp)) = make_uint4(b[4], b[5], b[6], b[7]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float2 fv = __half22float2(*reinterpret_cast<const __half2 *>(&r[i]));
+            sx += fv.x + fv.y;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    if (lane == 0) reinterpret_cast<float *>(meta)[m] = sx;
+}
+
+__global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
+    extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
+    const DkLayout lay(a.maxM, a.chained);
+    const int NS = (int)lay.ns;
+    // 1024-byte alignment for the 128-byte swizzle of the weight boxes
+    uint8_t *smem = dk_smem_raw + ((1024u - (smem_u32(dk_smem_raw) & 1023u)) & 1023u);
+    uint8_t *wring = smem + lay.w_off;
+    uint8_t *rawx = smem + lay.raw_off;
+    uint8_t *sslot = smem + lay.st_off;  // per slot: [meta 64 B][B operands]
+    uint8_t *parts = smem + lay.part_off;
+    DkQEntry *queue = reinterpret_cast<DkQEntry *>(smem + lay.q_off);
+    uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + lay.bar_off);  // copies landed
+    uint64_t *xfull = wfull + NS;                                         // stager -> consumers
+    uint64_t *empty = xfull + NS;                                         // consumers -> producer
+    uint64_t *qfull = empty + NS;
+    uint64_t *qempty = qfull + kDkQueue;
+    uint64_t *pfull = qempty + kDkQueue;  // consumers -> epilogue
+    uint64_t *pempty = pfull + kDkPartBufs;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&wfull[i], 1);
+            mbar_init(&xfull[i], 32);  // every stager lane arrives
+            mbar_init(&empty[i], kDkConsumers);
+        }
+        for (int i = 0; i < kDkQueue; ++i) {
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], kDkConsumers + kDkStagers + kDkEpilogues);
+        }
+        for (int i = 0; i < kDkPartBufs; ++i) {
+            mbar_init(&pfull[i], kDkConsumers);
+            mbar_init(&pempty[i], 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    if (warp != 0) {
+        // ---- every warp but the producer: convert activations, one unit at a time ----
+        pdl_wait();  // X may be written by the preceding grid; Y may still be in use
+        while (true) {
+            int u = 0;
+            if (lane == 0) u = (int)atomicAdd(&a.ctr[kDkCtrUnits], 1u);
+            u = __shfl_sync(0xffffffffu, u, 0);
+            if (u >= a.total_units) break;
+            const DkUnitRec U = dk_load_rec<DkUnitRec, 3>(a.units, u);
+            const int valid = min(U.K - U.stage * kDkStageTrits, kDkStageTrits);
+            const uint16_t *src = U.X + (int64_t)U.m * U.ldx + (int64_t)U.stage * kDkStageTrits;
+            if (U.M <= kDkImmaMaxM)
+                dk_conv_imma(src, valid, U.m, U.M, U.dst + kDkMetaBytes, U.dst, lane);
+            else
+                dk_conv_hmma(src, valid, U.m, U.M + (U.M & 1), U.dst + kDkMetaBytes, U.dst, lane);
+            // the converted unit is read by bulk copies of other CTAs
+            dk_fence_proxy_global();
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                atomicAdd(&a.ready[U.layer], 1u);
+                atomicAdd(&a.ctr[kDkCtrUnitsDone], 1u);
+            }
+        }
+    }
+
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        // Items are handed out dynamically: the first one is blockIdx.x, each
+        // later one comes from the workspace counter (plus gridDim.x).  The
+        // index of the item after next and the record of the next item are
+        // fetched while the current item streams.
+        uint32_t stage = 0;
+        int ps = 0;
+        uint32_t pph = 0;
+        bool wrapped = false;
+        int qi = 0;
+        bool waited = false, ok = true, all_ready = a.total_units == 0;
+        uint32_t final_seen = 0;
+        const int G = (int)gridDim.x;
+        int item = (int)blockIdx.x;
+        DkItemRec R{};
+        if (item < a.total_items) R = dk_load_rec<DkItemRec, 6>(a.items, item);
+        int next = a.total_items;
+        while (ok) {
+            const int q = qi % kDkQueue;
+            if (qi >= kDkQueue && !dk_warp_wait(&qempty[q], (uint32_t)((qi / kDkQueue) - 1) & 1u)) {
+                ok = false;
+                break;
+            }
+            const bool valid = item < a.total_items;
+            const bool pre = valid && R.B != nullptr;
+            if (lane == 0) {
+                DkQEntry e{};
+                e.item = valid ? item : -1;
+                if (valid) {
+                    e.Y = R.Y;
+                    e.part_off = R.part_off;
+                    e.alpha = R.alpha;
+                    e.tile = R.tile;
+                    e.part = R.part;
+                    e.s0 = R.s0;
+                    e.s1 = R.s1;
+                    e.M = R.M;
+                    e.K = R.K;
+                    e.N = R.N;
+                    e.ldy = R.ldy;
+                    e.parts = R.parts;
+                    e.tile_begin = R.tile_begin;
+                    e.pre = pre ? 1 : 0;
+                }
+                queue[q] = e;
+                mbar_arrive(&qfull[q]);
+            }
+            ++qi;
+            if (!valid) break;
+            const CUtensorMap *tmap = a.maps + R.layer;
+            const int n0 = R.tile * kDkRows;
+            // activation bytes of stage s for one token (whole 16-byte units)
+            auto xbytes = [&](int s) -> uint32_t {
+                const int rem = R.K - s * kDkStageTrits;
+                const int n = rem < kDkStageTrits ? ((rem + 7) & ~7) : kDkStageTrits;
+                return 2u * (uint32_t)n;
+            };
+            // bytes of a stage besides the weights
+            auto extra = [&](int s) -> uint32_t {
+                return pre ? (uint32_t)R.bstride : (uint32_t)R.M * xbytes(s);
+            };
+            auto issue_w = [&](int slot, int s) {
+                tma_load_2d(wring + slot * kDkWBytes, tmap, &wfull[slot], s * kDkStageW, n0);
+                tma_load_2d(wring + slot * kDkWBytes + kDkBoxBytes, tmap, &wfull[slot],
+                            s * kDkStageW + kDkSegBytes, n0);
+            };
+            auto issue_x = [&](int slot, int s) {
+                if (pre) {
+                    dk_bulk_load(sslot + slot * lay.slot_b, R.B + (int64_t)s * R.bstride,
+                                 (uint32_t)R.bstride, &wfull[slot]);
+                } else {
+                    const uint32_t b = xbytes(s);
+                    for (int m = 0; m < R.M; ++m)
+                        dk_bulk_load(rawx + slot * lay.raw_stage + m * kDkRawTok,
+                                     R.X + (int64_t)m * R.ldx + (int64_t)s * kDkStageTrits, b,
+                                     &wfull[slot]);
+                }
+            };
+            // the item's activations may be read: the layer's units are
+            // converted, or (chained layers) the earlier layers' outputs are final
+            auto wait_inputs = [&]() -> bool {
+                bool good = true;
+                if (pre) {
+                    if (!all_ready)
+                        good = dk_wait_count(&a.ready[R.layer], (uint32_t)R.need,
+                                             &a.ctr[kDkCtrUnitsDone], (uint32_t)a.total_units,
+                                             &all_ready);
+                } else if (R.wait_tiles > 0 && final_seen < (uint32_t)R.wait_tiles) {
+                    good = dk_wait_count(&a.ctr[kDkCtrFinal], (uint32_t)R.wait_tiles, nullptr, 0u,
+                                         nullptr);
+                    if (good) final_seen = (uint32_t)R.wait_tiles;
+                }
+                dk_fence_proxy_global();
+                return good;
+            };
+            int s = R.s0;
+            if (!waited) {
+                // first item: weights of up to a ring's worth of stages before the
+                // previous grid ends (expected bytes raised now, the arrival later)
+                const int pre_n = min(R.s1 - R.s0, NS);
+                if (lane == 0) {
+                    tma_prefetch_desc(tmap);
+                    for (int i = 0; i < pre_n; ++i) {
+                        const int slot = (int)((stage + i) % NS);
+                        dk_expect_tx(&wfull[slot], kDkWBytes);
+                        issue_w(slot, R.s0 + i);
+                    }
+                }
+                pdl_wait();
+                waited = true;
+                // the counter was reset by the previous grid's last CTA
+                int nx = 0;
+                if (lane == 0) nx = G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
+                next = __shfl_sync(0xffffffffu, nx, 0);
+                const bool in_ok = wait_inputs();
+                if (lane == 0) {
+                    for (int i = 0; i < pre_n; ++i) {
+                        const int slot = (int)((stage + i) % NS);
+                        const int si = R.s0 + i;
+                        mbar_arrive_expect_tx(&wfull[slot], in_ok ? extra(si) : 0u);
+                        if (in_ok) issue_x(slot, si);
+                    }
+                }
+                __syncwarp();
+                stage += pre_n;
+                s += pre_n;
+                ps = pre_n;
+                if (ps == NS) {
+                    ps = 0;
+                    pph = 1;
+                    wrapped = true;
+                }
+                if (!in_ok) {
+                    ok = false;
+                    break;
+                }
+            } else if (!wait_inputs()) {
+                ok = false;
+                break;
+            }
+            // fetched now, used after this item's stages are issued
+            DkItemRec NR{};
+            if (next < a.total_items) NR = dk_load_rec<DkItemRec, 6>(a.items, next);
+            int nx2 = 0;
+            if (lane == 0 && next < a.total_items)
+                nx2 = G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
+            for (; s < R.s1; ++s, ++stage) {
+                const int slot = ps;
+                if (wrapped && !dk_warp_wait(&empty[slot], pph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                if (++ps == NS) {
+                    ps = 0;
+                    pph ^= 1u;
+                    wrapped = true;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&wfull[slot], kDkWBytes + extra(s));
+                    issue_w(slot, s);
+                    issue_x(slot, s);
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            item = next;
+            R = NR;
+            next = next < a.total_items ? __shfl_sync(0xffffffffu, nx2, 0) : a.total_items;
+            if (item < a.total_items && lane == 0) tma_prefetch_desc(a.maps + R.layer);
+        }
+        if (!waited) pdl_wait();
+        // the CTA may not exit with copies still landing in its shared memory
+        for (uint32_t t = stage > (uint32_t)NS ? stage - NS : 0; t < stage; ++t)
+            mbar_wait(&wfull[t % NS], (t / NS) & 1u);
+    } else if (warp < kDkFirstEpi) {
+        // ---------------- stagers ----------------
+        // Converted stages only need their arrival; per-item stages (chained
+        // layers) are converted here from the raw activations.  Either way the
+        // stager first waits for the stage's copies, so xfull never runs a
+        // round ahead of the consumers.
+        const int sw = warp - 1;
+        int ss = 0;
+        uint32_t sph = 0;
+        int qi = 0;
+        bool ok = true;
+        DkQEntry e;
+        while (ok && dk_next_item(queue, qfull, qempty, qi, e)) {
+            const int M = e.M, K = e.K;
+            for (int s = e.s0; s < e.s1; ++s) {
+                const int slot = ss;
+                const uint32_t ph = sph;
+                if (++ss == NS) {
+                    ss = 0;
+                    sph ^= 1u;
+                }
+                if (slot % kDkStagers != sw) continue;  // another stager's slot
+                if (!dk_warp_wait(&wfull[slot], ph)) {
+                    ok = false;
+                    break;
+                }
+                if (!e.pre) {
+                    const int valid = min(K - s * kDkStageTrits, kDkStageTrits);
+                    uint8_t *dst = sslot + slot * lay.slot_b;
+                    for (int m = 0; m < M; ++m) {
+                        const uint16_t *src = reinterpret_cast<const uint16_t *>(
+                            rawx + slot * lay.raw_stage + m * kDkRawTok);
+                        if (M <= kDkImmaMaxM)
+                            dk_conv_imma(src, valid, m, M, dst + kDkMetaBytes, dst, lane);
+                        else
+                            dk_conv_hmma(src, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
+                    }
+                }
+                mbar_arrive(&xfull[slot]);
+            }
+        }
+    } else if (warp < kDkFirstCons) {
+        // ---------------- epilogues: warp 4 + i takes the items i, i + 2, ... ----------------
+        const int ew = warp - kDkFirstEpi;
+        int qi = 0, pi = -1;
+        DkQEntry e;
+        while (dk_next_item(queue, qfull, qempty, qi, e)) {
+            if (++pi % kDkEpilogues != ew) continue;
+            const int b = pi % kDkPartBufs;
+            if (!dk_warp_wait(&pfull[b], (uint32_t)(pi / kDkPartBufs) & 1u)) break;
+            const uint8_t *pb = parts + b * lay.parts;
+            const int M = e.M, n0 = e.tile * kDkRows, cnt = kDkRows * M;
+            const bool exact = M <= kDkImmaMaxM;
+            int64_t *slot = e.parts > 1 ? a.partials + e.part_off +
+                                              (int64_t)(e.tile * e.parts + e.part) * cnt
+                                        : nullptr;
+            // partial of (token m, warp cw, tile t, MMA row rho) at ((m*16 + cw)*2 + t)*16 + rho;
+            // the four warps of a row tile (cw, cw + 4, +8, +12) are 128 entries
+            // apart, and 32 consecutive rows of one token read 32 consecutive entries
+            for (int idx = lane; idx < cnt; idx += 32) {
+                const int r = idx % kDkRows, m = idx / kDkRows;  // consecutive lanes: consecutive n
+                const int t = r >> 4, tp = t >> 1, tl = t & 1;
+                const int rho = (r & 8) + dk_pi_inv(r & 7);
+                const int base = ((m * 16 + tp) * 2 + tl) * 16 + rho;
+                if (exact) {
+                    const int64_t *p = reinterpret_cast<const int64_t *>(pb);
+                    const int64_t v = p[base] + p[base + 128] + p[base + 256] + p[base + 384];
+                    if (slot) {
+                        slot[idx] = v;
+                    } else if (n0 + r < e.N) {
+                        const double y = (double)e.alpha * ((double)v * 5.9604644775390625e-8);
+                        e.Y[(int64_t)m * e.ldy + n0 + r] = __half_as_ushort(__double2half(y));
+                    }
+                } else {
+                    const float *p = reinterpret_cast<const float *>(pb);
+                    const float v = ((p[base] + p[base + 128]) + p[base + 256]) + p[base + 384];
+                    if (slot) {
+                        reinterpret_cast<double *>(slot)[idx] = (double)v;
+                    } else if (n0 + r < e.N) {
+                        e.Y[(int64_t)m * e.ldy + n0 + r] = f32_to_f16_bits(e.alpha * v);
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pempty[b]);
+            bool final_tile = true;
+            if (slot) {
+                __threadfence();
+                __syncwarp();
+                uint32_t prev = 0;
+                if (lane == 0) prev = atomicAdd(&a.tile_ctr[e.tile_begin + e.tile], 1u);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                final_tile = prev == (uint32_t)(e.parts - 1);
+                if (final_tile) {
+                    // last part of the tile: add the parts in part order
+                    __threadfence();
+                    const int64_t *base = a.partials + e.part_off + (int64_t)e.tile * e.parts * cnt;
+                    for (int i0 = 0; i0 < cnt; i0 += 32 * 4) {
+                        if (exact) {
+                            int64_t acc[4] = {0, 0, 0, 0};
+                            for (int q = 0; q < e.parts; ++q) {
+#pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const int idx = i0 + lane + 32 * t;
+                                    if (idx < cnt)
+                                        acc[t] += __ldcg(reinterpret_cast<const long long *>(
+                                            base + (int64_t)q * cnt + idx));
+                                }
+                            }
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int idx = i0 + lane + 32 * t;
+                                const int r = idx % kDkRows, m = idx / kDkRows;
+                                if (idx < cnt && n0 + r < e.N)
+                                    e.Y[(int64_t)m * e.ldy + n0 + r] = __half_as_ushort(__double2half(
+                                        (double)e.alpha * ((double)acc[t] * 5.9604644775390625e-8)));
+                            }
+                        } else {
+                            double acc[4] = {0.0, 0.0, 0.0, 0.0};
+                            for (int q = 0; q < e.parts; ++q) {
+#pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const int idx = i0 + lane + 32 * t;
+                                    if (idx < cnt)
+                                        acc[t] += __ldcg(reinterpret_cast<const double *>(
+                                            base + (int64_t)q * cnt + idx));
+                                }
+                            }
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int idx = i0 + lane + 32 * t;
+                                const int r = idx % kDkRows, m = idx / kDkRows;
+                                if (idx < cnt && n0 + r < e.N)
+                                    e.Y[(int64_t)m * e.ldy + n0 + r] =
+                                        f32_to_f16_bits(e.alpha * (float)acc[t]);
+                            }
+                        }
+                    }
+                    if (lane == 0) a.tile_ctr[e.tile_begin + e.tile] = 0u;
+                }
+            }
+            if (final_tile) {
+                // the tile's outputs are stored: count it for layers that read them
+                // (by bulk copies, through the async proxy)
+                dk_fence_proxy_global();
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicAdd(&a.ctr[kDkCtrFinal], 1u);
+            }
+        }
+    } else {
+        // ---------------- consumers ----------------
+        const int cw = warp - kDkFirstCons;
+        const int tp = cw & 3, qv = cw >> 2;
+        const int h = qv >> 1, v = qv & 1;
+        const int g = lane >> 2, c = lane & 3;
+        const int pg = dk_pi(g);
+        // tile 2tp, MMA row g: physical row 32 tp + pg; the 4 rows of this lane
+        // (tiles 2tp / 2tp+1, rows g / g+8) are 8 rows apart
+        const uint32_t aoff = (uint32_t)((32 * tp + pg) * kDkSegBytes + (((4 * v + c) ^ pg) << 4)) +
+                              (uint32_t)h * kDkBoxBytes;
+        int cs = 0;
+        uint32_t cph = 0;
+        int qi = 0, pi = 0;
+        bool ok = true;
+        DkQEntry e;
+        // waits for the stage's copies and conversion; false on a timeout
+        auto wait_stage = [&](int slot) -> bool {
+            return dk_warp_wait(&wfull[slot], cph) && dk_warp_wait(&xfull[slot], cph);
+        };
+        auto release = [&](int slot) {
+            // the shared-memory values are consumed (in registers) before the release
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (++cs == NS) {
+                cs = 0;
+                cph ^= 1u;
+            }
+        };
+        while (ok && dk_next_item(queue, qfull, qempty, qi, e)) {
+            const int M = e.M;
+            const int b = pi % kDkPartBufs;
+            uint8_t *pb = parts + b * lay.parts;
+            if (M == 1) {
+                // ---- integer engine, one token: one accumulator per digit
+                // position j (A = digits * 4^j, one AND per register) ----
+                int acc[2][4][4];  // [tile][digit position][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[t][j][0] = acc[t][j][1] = acc[t][j][2] = acc[t][j][3] = 0;
+                int64_t qsum = 0;
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A00 = dk_lds128(wb);                     // tile 2tp, row g
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);   // tile 2tp, row g + 8
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);  // tile 2tp + 1, row g
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);  // tile 2tp + 1, row g + 8
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    qsum += reinterpret_cast<const int64_t *>(sb)[0];
+                    const uint8_t *xg = sb + kDkMetaBytes + h * 4096 + ((v * 32 + g) * 4 + c) * 16;
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const int i0 = 2 * pr, i1 = i0 + 1;
+                        const uint4 B0 = dk_lds128(xg + i0 * 512), B1 = dk_lds128(xg + i1 * 512);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t m = 0x03030303u << (2 * j);
+                            const uint32_t b0 = dk_word(B0, j), b1 = dk_word(B1, j);
+                            mma_u8_16832(acc[0][j], dk_word(A00, i0) & m, dk_word(A01, i0) & m,
+                                         dk_word(A00, i1) & m, dk_word(A01, i1) & m, b0, b1);
+                            mma_u8_16832(acc[1][j], dk_word(A10, i0) & m, dk_word(A11, i0) & m,
+                                         dk_word(A10, i1) & m, dk_word(A11, i1) & m, b0, b1);
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= kDkPartBufs &&
+                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                    break;
+                // V = sum_p 256^p S_p - 2^40 S_ones - Q; this lane holds columns
+                // 2c, 2c + 1 (planes 2c, 2c + 1, or the ones column at c = 3)
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        int64_t d[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int q = 2 * rr + u;  // digit positions carry 4^j, exactly divisible
+                            d[u] = (int64_t)(acc[t][0][q] + (acc[t][1][q] >> 2) + (acc[t][2][q] >> 4) +
+                                             (acc[t][3][q] >> 6));
+                        }
+                        int64_t v0 = c < 3 ? (d[0] << (16 * c)) + (d[1] << (16 * c + 8)) : -(d[0] << 40);
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+                        if (qv == 0) v0 -= qsum;
+                        if (c == 0) reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                    }
+                }
+            } else if (M == 2) {
+                // ---- integer engine, two tokens: two column groups share the
+                // decoded digits (shifted to the low bits, one accumulator) ----
+                int iacc[2][2][4];  // [tile][column group][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
+                int64_t qsum0 = 0, qsum1 = 0;
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A00 = dk_lds128(wb);
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
+                    qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
+                    const uint8_t *xg = sb + kDkMetaBytes + h * 4096 + ((v * 32 + g) * 4 + c) * 16;
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        const int i0 = 2 * pr, i1 = i0 + 1;
+                        const uint4 B00 = dk_lds128(xg + i0 * 512), B01 = dk_lds128(xg + i1 * 512);
+                        const uint4 B10 = dk_lds128(xg + 8192 + i0 * 512);
+                        const uint4 B11 = dk_lds128(xg + 8192 + i1 * 512);
+#pragma unroll 2
+                        for (int j = 0; j < 4; ++j) {
+                            constexpr uint32_t m = 0x03030303u;
+                            const uint32_t a00 = (dk_word(A00, i0) >> (2 * j)) & m;
+                            const uint32_t a01 = (dk_word(A01, i0) >> (2 * j)) & m;
+                            const uint32_t a02 = (dk_word(A00, i1) >> (2 * j)) & m;
+                            const uint32_t a03 = (dk_word(A01, i1) >> (2 * j)) & m;
+                            const uint32_t a10 = (dk_word(A10, i0) >> (2 * j)) & m;
+                            const uint32_t a11 = (dk_word(A11, i0) >> (2 * j)) & m;
+                            const uint32_t a12 = (dk_word(A10, i1) >> (2 * j)) & m;
+                            const uint32_t a13 = (dk_word(A11, i1) >> (2 * j)) & m;
+                            const uint32_t b00 = dk_word(B00, j), b01 = dk_word(B01, j);
+                            const uint32_t b10 = dk_word(B10, j), b11 = dk_word(B11, j);
+                            mma_u8_16832(iacc[0][0], a00, a01, a02, a03, b00, b01);
+                            mma_u8_16832(iacc[1][0], a10, a11, a12, a13, b00, b01);
+                            mma_u8_16832(iacc[0][1], a00, a01, a02, a03, b10, b11);
+                            mma_u8_16832(iacc[1][1], a10, a11, a12, a13, b10, b11);
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= kDkPartBufs &&
+                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                    break;
+                // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
+                // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int64_t d0 = iacc[t][0][2 * rr], d1 = iacc[t][0][2 * rr + 1];
+                        const int64_t e0 = iacc[t][1][2 * rr], e1 = iacc[t][1][2 * rr + 1];
+                        int64_t v0 = 0, v1 = 0;
+                        if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
+                        else v1 = d0 + (d1 << 8);
+                        if (c < 2) {
+                            v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
+                        } else if (c == 2) {
+                            v0 -= e0 << 40;
+                            v1 -= e0 << 40;
+                        }
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+                        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+                        if (qv == 0) {
+                            v0 -= qsum0;
+                            v1 -= qsum1;
+                        }
+                        if (c == 0) {
+                            int64_t *p = reinterpret_cast<int64_t *>(pb);
+                            p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                            p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
+                        }
+                    }
+                }
+            } else {
+                // ---- fp16 engine ----
+                const int Mp = M + (M & 1);
+                float facc[2][4][4];  // [tile][digit position][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        facc[t][q][0] = facc[t][q][1] = facc[t][q][2] = facc[t][q][3] = 0.f;
+                float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A00 = dk_lds128(wb);
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    const float *mt = reinterpret_cast<const float *>(sb);
+                    if (2 * c < M) sx0 += mt[2 * c];
+                    if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
+                    const uint8_t *xb = sb + kDkMetaBytes;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 B0 = make_uint4(0u, 0u, 0u, 0u), B1 = B0;
+                        if (g < M) {
+                            const int w = h * 32 + (4 * v + c) * 4 + i;
+                            B0 = dk_lds128(xb + dk_hblock(w, g, 0, Mp));
+                            B1 = dk_lds128(xb + dk_hblock(w, g, 1, Mp));
+                        }
+                        const uint32_t bb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
+                        const uint32_t W0 = dk_word(A00, i), V0 = dk_word(A01, i);
+                        const uint32_t W1 = dk_word(A10, i), V1 = dk_word(A11, i);
+                        const uint32_t hW0 = W0 >> 8, hV0 = V0 >> 8, hW1 = W1 >> 8, hV1 = V1 >> 8;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t m = 0x00030003u << (2 * j);
+                            mma_16816(facc[0][j], W0 & m, V0 & m, hW0 & m, hV0 & m, bb[2 * j],
+                                      bb[2 * j + 1]);
+                            mma_16816(facc[1][j], W1 & m, V1 & m, hW1 & m, hV1 & m, bb[2 * j],
+                                      bb[2 * j + 1]);
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= kDkPartBufs &&
+                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                    break;
+                float *p = reinterpret_cast<float *>(pb);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    float sv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        sv[q] = facc[t][0][q] * 16777216.0f + facc[t][1][q] * 4194304.0f +
+                                facc[t][2][q] * 1048576.0f + facc[t][3][q] * 262144.0f;
+                    if (qv == 0) {
+                        sv[0] -= sx0;
+                        sv[1] -= sx1;
+                        sv[2] -= sx0;
+                        sv[3] -= sx1;
+                    }
+                    const int m0 = 2 * c, m1 = 2 * c + 1;
+                    if (m0 < M) {
+                        p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
+                        p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
+                    }
+                    if (m1 < M) {
+                        p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
+                        p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pfull[b]);
+            ++pi;
+        }
+    }
+
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // the last CTA out leaves the workspace counters at zero for the next launch
+        __threadfence();
+        const uint32_t done = atomicAdd(&a.ctr[kDkCtrDone], 1u);
+        if (done == gridDim.x - 1) {
+            __threadfence();
+            a.ctr[kDkCtrFinal] = 0u;
+            a.ctr[kDkCtrItems] = 0u;
+            a.ctr[kDkCtrUnits] = 0u;
+            a.ctr[kDkCtrUnitsDone] = 0u;
+            for (int l = 0; l < a.count; ++l) a.ready[l] = 0u;
+            a.ctr[kDkCtrDone] = 0u;
+        }
+    }
+}
+
+}  // namespace tlk
+
+// ---- host side ---------------------------------------------------------------
+namespace tlk {
+
+// K-parts of a layer: items of about kDkItemStages stages, cut at stage
+// boundaries, never more than kDkMaxItemStages stages per item.
+inline int dk_parts(int stages) {
+    int parts = (stages + kDkItemStages / 2) / kDkItemStages;
+    if (parts < 1) parts = 1;
+    while ((stages + parts - 1) / parts > kDkMaxItemStages) ++parts;
+    if (parts > stages) parts = stages;
+    return parts;
+}
+
+struct DkHostLayer {
+    const uint8_t *T;
+    const uint16_t *X;
+    uint16_t *Y;
+    int64_t ldp, ldx, ldy;
+    float alpha;
+    int M, N, K;
+    bool reads_earlier;
+};
+
+struct DkSchedule {
+    int count = 0, total_items = 0, total_units = 0, total_tiles = 0, maxM = 1, chained = 0;
+    int64_t slots = 0, staged = 0;
+    size_t bytes = 0;
+};
+
+// Sizes of a batch; with `items` and `units` given, also their tables, holding
+// pointers into the workspace at `ws`.  Items are in layer order, then tile,
+// then part; units in layer order, then stage, then token.
+inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
+                              std::vector<DkItemRec> *items, std::vector<DkUnitRec> *units) {
+    DkSchedule sc;
+    sc.count = count;
+    for (int l = 0; l < count; ++l) {
+        const DkHostLayer &h = in[l];
+        const int stages = (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
+        const int parts = dk_parts(stages);
+        const int tiles = (h.N + kDkRows - 1) / kDkRows;
+        sc.total_items += tiles * parts;
+        sc.total_tiles += tiles;
+        if (h.reads_earlier) {
+            sc.chained = 1;
+        } else {
+            sc.total_units += stages * h.M;
+            sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(h.M));
+        }
+        if (parts > 1) sc.slots += (int64_t)tiles * parts * kDkRows * h.M;
+        if (h.M > sc.maxM) sc.maxM = h.M;
+    }
+    const DkWsLayout wl(count, sc.total_items, sc.total_units, sc.total_tiles, sc.slots, sc.staged);
+    sc.bytes = wl.total;
+    if (!items || !units) return sc;
+    int64_t slots = 0, staged = 0;
+    int tile_begin = 0;
+    for (int l = 0; l < count; ++l) {
+        const DkHostLayer &h = in[l];
+        const int stages = (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
+        const int parts = dk_parts(stages);
+        const int tiles = (h.N + kDkRows - 1) / kDkRows;
+        const int bstride = kDkMetaBytes + (int)dk_stage_b(h.M);
+        uint8_t *B = h.reads_earlier ? nullptr : ws + wl.staged + staged;
+        for (int t = 0; t < tiles; ++t)
+            for (int q = 0; q < parts; ++q) {
+                DkItemRec r{};
+                r.X = h.X;
+                r.Y = h.Y;
+                r.B = B;
+                r.part_off = slots;
+                r.alpha = h.alpha;
+                r.layer = l;
+                r.tile = t;
+                r.part = q;
+                r.s0 = (int)((int64_t)stages * q / parts);
+                r.s1 = (int)((int64_t)stages * (q + 1) / parts);
+                r.M = h.M;
+                r.K = h.K;
+                r.N = h.N;
+                r.ldx = (int)h.ldx;
+                r.ldy = (int)h.ldy;
+                r.parts = parts;
+                r.tile_begin = tile_begin;
+                r.wait_tiles = h.reads_earlier ? tile_begin : 0;
+                r.need = stages * h.M;
+                r.bstride = bstride;
+                items->push_back(r);
+            }
+        if (B)
+            for (int s = 0; s < stages; ++s)
+                for (int m = 0; m < h.M; ++m) {
+                    DkUnitRec u{};
+                    u.X = h.X;
+                    u.dst = B + (int64_t)s * bstride;
+                    u.layer = l;
+                    u.stage = s;
+                    u.m = m;
+                    u.M = h.M;
+                    u.K = h.K;
+                    u.ldx = (int)h.ldx;
+                    units->push_back(u);
+                }
+        if (parts > 1) slots += (int64_t)tiles * parts * kDkRows * h.M;
+        if (B) staged += (int64_t)stages * bstride;
+        tile_begin += tiles;
+    }
+    return sc;
+}
+
+// Tensor map of a layer's packed weights: bytes x rows, boxes of 128 bytes x
+// 128 rows with the 128-byte swizzle, zero fill outside [0, row bytes) x [0, N).
+inline bool dk_encode_map(const DkHostLayer &h, CUtensorMap *map) {
+    auto encode = tensor_map_encoder();
+    if (!encode) return false;
+    const int64_t rowbytes = ((int64_t)h.K + 3) / 4;
+    cuuint64_t dims[2] = {(cuuint64_t)rowbytes, (cuuint64_t)h.N};
+    cuuint64_t strides[1] = {(cuuint64_t)h.ldp};
+    cuuint32_t box[2] = {(cuuint32_t)kDkSegBytes, (cuuint32_t)kDkRows};
+    cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(h.T), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int total_tiles,
+                      int maxM, int chained) {
+    const DkWsLayout wl(count, total_items, total_units, total_tiles, 0, 0);
+    uint8_t *b = reinterpret_cast<uint8_t *>(ws);
+    DkArgs a;
+    a.ctr = reinterpret_cast<uint32_t *>(b);
+    a.maps = reinterpret_cast<const CUtensorMap *>(b + wl.maps);
+    a.items = reinterpret_cast<const DkItemRec *>(b + wl.items);
+    a.units = reinterpret_cast<const DkUnitRec *>(b + wl.units);
+    a.ready = reinterpret_cast<uint32_t *>(b + wl.ready);
+    a.tile_ctr = reinterpret_cast<uint32_t *>(b + wl.tiles);
+    a.partials = reinterpret_cast<int64_t *>(b + wl.partials);
+    a.count = count;
+    a.total_items = total_items;
+    a.total_units = total_units;
+    a.maxM = maxM;
+    a.chained = chained;
+    return a;
+}
+
+inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t stream,
+                          int *last_cuda_error) {
+    constexpr int kMaxDev = 64;
+    static std::once_flag once[kMaxDev];
+    static cudaError_t attr_err[kMaxDev];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDev) {
+        *last_cuda_error = (int)e;
+        return 5;
+    }
+    std::call_once(once[dev], [dev] {
+        uint32_t most = 0;
+        for (int m = 1; m <= 8; ++m) {
+            const uint32_t t = DkLayout(m, 1).total;
+            most = t > most ? t : most;
+        }
+        attr_err[dev] = cudaFuncSetAttribute(decode2_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+    });
+    if (attr_err[dev] != cudaSuccess) {
+        *last_cuda_error = (int)attr_err[dev];
+        return 5;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.total_items < num_sms ? a.total_items : num_sms));
+    cfg.blockDim = dim3(kDkThreads);
+    cfg.dynamicSmemBytes = DkLayout(a.maxM, a.chained).total;
+    cfg.stream = stream;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, decode2_kernel, a);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        *last_cuda_error = (int)e;
+        return 5;
+    }
+    return 0;
+}
+
+}  // namespace tlk

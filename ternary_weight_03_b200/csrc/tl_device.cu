@@ -1,6 +1,7 @@
 // tl_device.cu -- device entry points of libternary: argument validation,
 // kernel selection and launch for tl_gemv / tl_gemm / tl_gemv_batch /
 // tl_ternarise, and the device error word behind tl_device_status.
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 #include <vector>
@@ -12,6 +13,7 @@
 #include "tl_gemm.cuh"
 #include "tl_gemv3.cuh"
 #include "tl_gemvp.cuh"
+#include "tl_decode.cuh"
 #include "tl_ternarise.cuh"
 
 namespace {
@@ -66,6 +68,10 @@ const DeviceInfo *device_info() {
     return &g_devices[dev];
 }
 
+// Per device: the number of the latest static plan (0: none yet).  A static
+// plan whose number is older describes a table that has been overwritten.
+std::atomic<uint64_t> g_static_generation[kMaxDevices];
+
 int gemv_occupancy(int fmt, int warps) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
@@ -106,6 +112,57 @@ int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::GpHostLay
         out[l] = tlk::GpHostLayer{a.dT, a.dX, a.dY, a.ldp, a.ldx, a.ldy, a.alpha, a.M, (int)a.N,
                                   (int)a.K, (a.flags & TL_LAYER_READS_EARLIER) != 0};
     }
+    return TL_OK;
+}
+
+// The 2-bit batch kernel's host layers (the same fields).
+std::vector<tlk::DkHostLayer> dk_layers(const std::vector<tlk::GpHostLayer> &h) {
+    std::vector<tlk::DkHostLayer> out(h.size());
+    for (size_t l = 0; l < h.size(); ++l)
+        out[l] = tlk::DkHostLayer{h[l].T, h[l].X, h[l].Y, h[l].ldp, h[l].ldx, h[l].ldy,
+                                  h[l].alpha, h[l].M, h[l].N, h[l].K, h[l].reads_earlier};
+    return out;
+}
+
+// tl_gemv_batch_plan for 2-bit layers (tl_decode.cuh): layer table, tensor
+// maps and zeroed counters written into the workspace.
+int plan_decode2(int count, const std::vector<tlk::GpHostLayer> &h, void *dWorkspace,
+                 size_t workspace_bytes, tl_gemv_plan *plan) {
+    std::vector<tlk::DkHostLayer> dh = dk_layers(h);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(dWorkspace);
+    std::vector<tlk::DkItemRec> items;
+    std::vector<tlk::DkUnitRec> units;
+    const tlk::DkSchedule sc = tlk::dk_schedule(count, dh.data(), ws, &items, &units);
+    if (sc.bytes > workspace_bytes) return TL_ERR_INVALID_ARG;
+    std::vector<CUtensorMap> maps(count);
+    for (int l = 0; l < count; ++l)
+        if (!tlk::dk_encode_map(dh[l], &maps[l])) return TL_ERR_CUDA;
+    if (!device_info()) return TL_ERR_CUDA;
+    const tlk::DkWsLayout wl(count, sc.total_items, sc.total_units, sc.total_tiles, sc.slots,
+                             sc.staged);
+    cudaError_t e = cudaMemset(ws, 0, wl.maps);  // counters
+    if (e == cudaSuccess)
+        e = cudaMemcpy(ws + wl.maps, maps.data(), sizeof(CUtensorMap) * count,
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(ws + wl.items, items.data(), sizeof(tlk::DkItemRec) * items.size(),
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && !units.empty())
+        e = cudaMemcpy(ws + wl.units, units.data(), sizeof(tlk::DkUnitRec) * units.size(),
+                       cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemset(ws + wl.ready, 0, wl.partials - wl.ready);  // ready, tiles
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e);
+    plan->fmt = TL_FMT_2BIT;
+    plan->count = count;
+    plan->max_m = sc.maxM;
+    plan->total_items = sc.total_items;
+    plan->total_tiles = sc.total_tiles;
+    plan->total_units = sc.total_units;
+    plan->chained = sc.chained;
+    plan->dWorkspace = dWorkspace;
+    plan->workspace_bytes = workspace_bytes;
+    plan->generation = 0;
     return TL_OK;
 }
 
@@ -193,6 +250,11 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
     std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
     int rc = batch_layers(fmt, count, layers, h.data());
     if (rc != TL_OK) return rc;
+    if (fmt == TL_FMT_2BIT) {
+        std::vector<tlk::DkHostLayer> dh = dk_layers(h);
+        *bytes = tlk::dk_schedule(count, dh.data(), nullptr, nullptr, nullptr).bytes;
+        return TL_OK;
+    }
     std::vector<tlk::GpLayer> table(count);
     *bytes = tlk::gp_schedule(fmt, count, h.data(), table.data()).bytes;
     return TL_OK;
@@ -205,6 +267,7 @@ int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dW
     std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
     int rc = batch_layers(fmt, count, layers, h.data());
     if (rc != TL_OK) return rc;
+    if (fmt == TL_FMT_2BIT) return plan_decode2(count, h, dWorkspace, workspace_bytes, plan);
     std::vector<tlk::GpLayer> table(count);
     const tlk::GpSchedule sc = tlk::gp_schedule(fmt, count, h.data(), table.data());
     if (sc.bytes > workspace_bytes) return TL_ERR_INVALID_ARG;
@@ -226,11 +289,14 @@ int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dW
     if (e != cudaSuccess) return cuda_fail(e);
     plan->fmt = fmt;
     plan->count = count;
+    plan->total_units = 0;
+    plan->chained = 0;
     plan->max_m = sc.maxM;
     plan->total_items = sc.total_items;
     plan->total_tiles = sc.total_tiles;
     plan->dWorkspace = dWorkspace;
     plan->workspace_bytes = workspace_bytes;
+    plan->generation = 0;
     return TL_OK;
 }
 
@@ -241,13 +307,23 @@ int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
     int rc = tl_gemv_batch_bytes(fmt, count, layers, &need);
     if (rc != TL_OK) return rc;
     if (need > (size_t)TL_STATIC_WORKSPACE_BYTES) return TL_ERR_INVALID_ARG;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return TL_ERR_INVALID_ARG;
     void *addr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&addr, g_static_workspace);  // this device's copy
+    e = cudaGetSymbolAddress(&addr, g_static_workspace);  // this device's copy
     if (e != cudaSuccess) return cuda_fail(e);
     // no run of an earlier static plan may still be reading the array
     e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e);
-    return tl_gemv_batch_plan(fmt, count, layers, addr, (size_t)TL_STATIC_WORKSPACE_BYTES, plan);
+    // every earlier static plan of this device is stale from here on, even if
+    // the rewrite below fails half way
+    const uint64_t gen = g_static_generation[dev].fetch_add(1) + 1;
+    rc = tl_gemv_batch_plan(fmt, count, layers, addr, (size_t)TL_STATIC_WORKSPACE_BYTES, plan);
+    if (rc != TL_OK) return rc;
+    plan->generation = gen;
+    return TL_OK;
 }
 
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream) {
@@ -255,13 +331,31 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
     if (flags & ~(unsigned int)TL_FLAG_PDL) return TL_ERR_INVALID_ARG;
     if (plan->fmt != TL_FMT_2BIT && plan->fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
     if (plan->count < 1 || plan->count > TL_GEMV_BATCH_MAX || plan->max_m < 1 ||
-        plan->max_m > TL_GEMV_MAX_M || plan->total_items < 1 || plan->total_tiles < 1)
+        plan->max_m > TL_GEMV_MAX_M || plan->total_items < 1 || plan->total_tiles < 1 ||
+        plan->total_units < 0 || (plan->chained != 0 && plan->chained != 1))
         return TL_ERR_INVALID_ARG;
     const DeviceInfo *dev = device_info();
     if (!dev) return TL_ERR_CUDA;
+    if (plan->generation != 0) {
+        // a static plan: only the device's latest, on the device that planned it
+        int d = 0;
+        cudaError_t e = cudaGetDevice(&d);
+        if (e != cudaSuccess) return cuda_fail(e);
+        void *addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_static_workspace);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (plan->dWorkspace != addr || plan->generation != g_static_generation[d].load())
+            return TL_ERR_INVALID_ARG;
+    }
+    const bool pdl = (flags & TL_FLAG_PDL) != 0;
+    if (plan->fmt == TL_FMT_2BIT) {
+        const tlk::DkArgs da =
+            tlk::dk_args(plan->dWorkspace, plan->count, plan->total_items, plan->total_units,
+                         plan->total_tiles, plan->max_m, plan->chained);
+        return tlk::launch_decode2(da, dev->num_sms, pdl, (cudaStream_t)stream, &t_last_cuda_error);
+    }
     const tlk::GpArgs a = tlk::gp_args(plan->dWorkspace, plan->count, plan->total_items,
                                        plan->total_tiles, plan->max_m);
-    const bool pdl = (flags & TL_FLAG_PDL) != 0;
     return plan->fmt == TL_FMT_2BIT
                ? tlk::launch_gemvp<2>(a, dev->num_sms, pdl, (cudaStream_t)stream,
                                       &t_last_cuda_error)

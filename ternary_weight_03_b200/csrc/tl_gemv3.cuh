@@ -319,6 +319,9 @@ gemv3_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restr
             if (n < N) Y[(int64_t)m * ldy + n] = f32_to_f16_bits(alpha * (acc - sx));
         }
     }
+    // no CTA leaves while a peer may still push into its shared memory (a peer
+    // whose own wait timed out above still gets here: every wait is bounded)
+    if (S > 1) cluster_sync();
 }
 
 // ---- host side ---------------------------------------------------------------

@@ -104,21 +104,51 @@ def _ws(L, fmt, arr):
     return rc, n.value
 
 
+def _up(v):
+    return (v + 255) // 256 * 256
+
+
+def _ws2_expected(layers):
+    """2-bit batch workspace, region by region (each rounded up to 256 bytes):
+    counters, one 128-byte tensor map per layer, a 96-byte record per work item
+    (128-row tile x K-part), a 48-byte record per conversion unit (stage x token
+    of a layer that reads no earlier output), a u32 per layer and per tile,
+    8-byte partials of split tiles, and the converted activations
+    (64 + 8 KB, 16 KB or 2 KB x even(M) bytes per stage)."""
+    items = units = tiles = slots = staged = 0
+    for d in layers:
+        stages = -(-(-(-d["K"] // 4)) // 256)
+        parts = max(1, min(stages, (stages + 2) // 4))
+        t = -(-d["N"] // 128)
+        items += t * parts
+        tiles += t
+        if not d.get("flags", 0):
+            units += stages * d["M"]
+            b = 8192 if d["M"] == 1 else (16384 if d["M"] == 2 else 2048 * (d["M"] + d["M"] % 2))
+            staged += stages * (64 + b)
+        if parts > 1:
+            slots += t * parts * 128 * d["M"]
+    off = 256
+    for size in (128 * len(layers), 96 * items, 48 * units, 4 * len(layers), 4 * tiles, 8 * slots,
+                 staged):
+        off = _up(off + size)
+    return off
+
+
 def test_batch_workspace_size(L):
-    # table (one 88-byte entry + one 128-byte TMA descriptor per layer), counters,
-    # and fp32 partials only for layers whose rows are split across CTAs
-    rc, n = _ws(L, 2, _layers([dict(N=1000, K=2048, ldp=512, ldx=2048, ldy=1000)]))
+    base = dict(M=1, flags=0)
+    cases = [[dict(base, N=1000, K=2048)], [dict(base, N=4096, K=14336)],
+             [dict(base, N=4096, K=14336, M=8)], [dict(base, N=4096, K=14336, M=2)],
+             [dict(base, N=130, K=700, M=3), dict(base, N=77, K=5000, M=1, flags=1)]]
+    for ls in cases:
+        arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16, ldx=d["K"] +
+                            (-d["K"]) % 8, ldy=d["N"] + (-d["N"]) % 8) for d in ls])
+        rc, n = _ws(L, 2, arr)
+        assert rc == 0 and n == _ws2_expected(ls), (ls, n)
+    # 1.6-bit: table (one 88-byte entry + one 128-byte TMA descriptor per layer),
+    # counters, and fp32 partials only for layers whose rows are split
+    rc, n = _ws(L, 16, _layers([dict(N=1000, K=2048, ldp=416, ldx=2048, ldy=1000)]))
     assert rc == 0 and n == 1024  # header 256, table 256, map 256, 9 tile counters 256
-    rc1, n1 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096, M=1)]))
-    rc8, n8 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096, M=8)]))
-    assert rc1 == rc8 == 0
-    tiles = (4096 + 119) // 120
-    assert n1 > 1024 and n8 > n1
-    # documented bound: ~200 B per layer + ~N * M * 4 * (K / 2048) for a split layer
-    assert n1 <= 2048 + 4096 * 1 * 4 * (14336 // 2048 + 1) * 128 // 120
-    rc2, n2 = _ws(L, 2, _layers([dict(N=4096, K=14336, ldp=3584, ldx=14336, ldy=4096,
-                                      dT=A + 4096)] * 2))
-    assert rc2 == 0 and n2 >= 2 * (n1 - 1024)
 
 
 @pytest.mark.parametrize("spec,count,rc", [
@@ -156,6 +186,9 @@ def test_batch_plan_and_run_rules(L):
     good = tl.Plan(fmt=2, count=2, max_m=1, total_items=3, total_tiles=2, dWorkspace=A,
                    workspace_bytes=n)
     assert L.tl_gemv_batch_run(ctypes.byref(good), 8, None) == 1   # unknown flag
+    bad_units = tl.Plan(fmt=2, count=2, max_m=1, total_items=3, total_tiles=2, total_units=-1,
+                        dWorkspace=A, workspace_bytes=n)
+    assert L.tl_gemv_batch_run(ctypes.byref(bad_units), 0, None) == 1
 
 
 def ternarise_rc(L, fmt=2, dW=A, ldw=1024, N=64, K=1024, dP=A, ldp=256, dAlpha=A, ws=A):

@@ -61,6 +61,26 @@ def test_static_workspace_matches_caller_workspace(fmt):
                 assert np.array_equal(a, b)
 
 
+def test_replaced_static_plan_is_rejected():
+    """A static plan made before a later tl_gemv_batch_plan_static describes a
+    table that has since been overwritten: running it returns
+    TL_ERR_INVALID_ARG without launching, and the newer plan still runs."""
+    import ternary_weight_03_b200 as tl
+    a = tl.make_layers(2, _batch(2, [(1, 500, 3000)], 600))
+    b_specs = _batch(2, [(8, 130, 4100), (2, 77, 700)], 700)
+    b = tl.make_layers(2, b_specs)
+    plan_a = tl.gemv_batch_plan_static(2, a)
+    plan_b = tl.gemv_batch_plan_static(2, b)
+    assert plan_a.generation != 0 and plan_b.generation != plan_a.generation
+    with pytest.raises(tl.TLError) as err:
+        tl.gemv_batch_run(plan_a)
+    assert err.value.status == 1
+    tl.gemv_batch_run(plan_b)
+    assert tl.device_status() == 0
+    for sp in b_specs:
+        assert not np.isnan(sp[4].float().cpu().numpy()[:, :sp[0].shape[0]]).any()
+
+
 def test_static_workspace_rejects_oversized_batch():
     import ctypes
     import ternary_weight_03_b200 as tl
