@@ -163,11 +163,11 @@ typedef struct tl_gemv_plan {
 } tl_gemv_plan;
 
 /* Workspace bytes a batch needs.  2-bit: counters, one TMA descriptor per
- * layer, a 96-byte record per work item (128 output rows x about 4096 trits
+ * layer, a 96-byte record per work item (256 output rows x 4096..8192 trits
  * of K), the layers' activations converted once into the tensor-core operand
- * layout (per 1024 trits of K: 8 KB at M = 1, 16 KB at M = 2, 2 KB per token
+ * layout (per 512 trits of K: 4 KB at M = 1, 8 KB at M = 2, 1 KB per token
  * rounded up to even at M >= 3, plus 64 B; none for TL_LAYER_READS_EARLIER
- * layers, which convert on chip) with a 48-byte record per 1024 trits and
+ * layers, which convert on chip) with a 48-byte record per 512 trits and
  * token, and 8-byte partial sums of rows split into K-parts (N * M * 8 bytes
  * per part).  1.6-bit: the layer table and one TMA descriptor per layer
  * (~200 B per layer), counters, and fp32 partial sums of the layers whose

@@ -5,7 +5,7 @@
 // Decoding streams every packed weight once and is bound by memory bandwidth
 // ("Pith review of Spectra 1.1", "What carries the argument"), so the kernel
 // is built around keeping HBM busy: one CTA per SM walks a queue of work
-// items (layer, 128-row tile, K-part) across all layers of the batch, and the
+// items (layer, 256-row tile, K-part) across all layers of the batch, and the
 // instructions spent per packed byte must stay far below what the SM can
 // issue.  Two tensor-core engines, chosen per item by its token count:
 //
@@ -27,31 +27,31 @@
 //    position, combined with exact power-of-two scales; sum_k x_k is
 //    subtracted at the end (d = t + 1).
 //
-// Weights arrive by TMA in 128-byte-wide boxes of 128 rows with the 128-byte
-// swizzle, two boxes per stage (256 packed bytes = 1024 trits per row).  A
-// consumer lane (g, c) reads 16-byte chunk 4v + c of rows g and g + 8 of a
-// 16-row tile; MMA row g is physical row pi(g) = ((g & 1) << 2) | (g >> 1), so
+// Weights arrive by TMA in boxes of 256 rows x 128 bytes (512 trits per row)
+// with the 128-byte swizzle, one box per stage.  A consumer lane (g, c) reads
+// 16-byte chunk 4v + c of rows g and g + 8 of a 16-row tile; MMA row g is physical row pi(g) = ((g & 1) << 2) | (g >> 1), so
 // the two rows of every quarter-warp differ in bit 2 and each LDS.128 touches
 // every bank once.
 //
 // Activations go into the B layout of their engine once per (layer, stage),
 // not once per item: every warp except the producer first converts such
-// units (handed out through a workspace counter) into the workspace and
-// counts them per layer; a stage's converted operands then arrive by one
+// units (unit u by converting warp u mod their number) into the workspace
+// and counts them per layer; a stage's converted operands then arrive by one
 // bulk copy next to its weights.  Layers flagged as reading an earlier
 // layer's output (their X is written during this launch) are converted per
-// item instead, from raw activations, by stager warps.
+// item instead, from X in global memory, by stager warps.
 //
-// Warp roles of a CTA (704 threads):
+// Warp roles of a CTA (768 threads):
 //  * warp 0, producer: issues each stage's copies into a ring and queues items
 //    (items come from a workspace counter, fetched one item ahead);
 //  * warps 1..3, stagers (warp 1 + i owns the ring slots s with s mod 3 = i);
-//  * warps 4, 5, epilogues (alternate items): sum the consumer partials of an
-//    item in a fixed order, then write Y, or a partial of a split tile to the
-//    workspace where the last part to arrive adds the parts in part order;
-//  * warps 6..21, consumers: warp w takes row tiles 2 (w & 3) and 2 (w & 3) + 1
-//    and the quarter w >> 2 of every stage (segment (w >> 3), chunks
-//    4 ((w >> 2) & 1) .. +3).
+//  * warps 4..7, epilogues (item i goes to warp 4 + i mod 4, or mod 2 when
+//    only two partial buffers fit): sum the consumer
+//    partials of an item in a fixed order, then write Y, or a partial of a
+//    split tile to the workspace where the last part to arrive adds the parts
+//    in part order;
+//  * warps 8..23, consumers: warp w takes row tiles 2 (w & 7) and 2 (w & 7) + 1
+//    and the half w >> 3 of every stage (chunks 4 (w >> 3) .. +3).
 // The cross-warp and cross-CTA sums follow the pages' shared-memory tree
 // reduction of per-warp partials (Figure 11 caption text on appendix G.4 of the
 // same page), in a fixed order.  All waits are bounded; a timeout sets the
@@ -59,6 +59,7 @@
 // they stay zero between launches.
 #pragma once
 #include <cuda.h>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -67,27 +68,25 @@
 
 namespace tlk {
 
-constexpr int kDkTiles = 8;                              // 16-row MMA tiles per item
-constexpr int kDkRows = 16 * kDkTiles;                   // 128 weight rows per item
-constexpr int kDkSegBytes = 128;                         // packed bytes per row per TMA box
-constexpr int kDkStageW = 2 * kDkSegBytes;               // packed bytes per row per stage
-constexpr int kDkStageTrits = 4 * kDkStageW;             // 1024 activations per stage
-constexpr int kDkBoxBytes = kDkRows * kDkSegBytes;       // 16 KB
-constexpr int kDkWBytes = 2 * kDkBoxBytes;               // 32 KB of weights per stage
-constexpr int kDkRawTok = 2 * kDkStageTrits;             // 2 KB of fp16 activations per token
+constexpr int kDkTiles = 16;                             // 16-row MMA tiles per item
+constexpr int kDkRows = 16 * kDkTiles;                   // 256 weight rows per item
+constexpr int kDkStageW = 128;                           // packed bytes per row per stage (one box)
+constexpr int kDkStageTrits = 4 * kDkStageW;             // 512 activations per stage
+constexpr int kDkWords = kDkStageW / 4;                  // 32 words of 16 trits per row per stage
+constexpr int kDkWBytes = kDkRows * kDkStageW;           // 32 KB of weights per stage
 constexpr int kDkConsumers = 16;
 constexpr int kDkStagers = 3;
-constexpr int kDkEpilogues = 2;
+constexpr int kDkEpilogues = 4;
 constexpr int kDkFirstEpi = 1 + kDkStagers;
 constexpr int kDkFirstCons = kDkFirstEpi + kDkEpilogues;
-constexpr int kDkWarps = kDkFirstCons + kDkConsumers;  // 22
-constexpr int kDkThreads = 32 * kDkWarps;              // 704
+constexpr int kDkWarps = kDkFirstCons + kDkConsumers;  // 24
+constexpr int kDkThreads = 32 * kDkWarps;              // 768
 constexpr int kDkMaxStages = 6;
 constexpr int kDkQueue = 16;
-constexpr int kDkPartBufs = 2;
+constexpr int kDkMaxPartBufs = 4;  // consumer -> epilogue buffers (2 when they are large)
 constexpr int kDkImmaMaxM = 2;                          // exact integer engine up to 2 tokens
-constexpr int kDkItemStages = 4;                        // target stages per item
-constexpr int kDkMaxItemStages = 32;                    // s32 sums of an item stay exact
+constexpr int kDkRefSms = 148;                          // scheduling reference: SMs of a B200
+constexpr int kDkMaxItemStages = 64;                    // s32 sums of an item stay exact
 constexpr uint32_t kDkSmemBudget = 232448u;             // 227 KB
 constexpr int kDkMetaBytes = 64;                        // per stage: per-token offsets, first
 
@@ -95,14 +94,13 @@ constexpr int kDkMetaBytes = 64;                        // per stage: per-token 
 constexpr int kDkCtrFinal = 1;      // tiles whose outputs are stored
 constexpr int kDkCtrDone = 2;       // CTAs that have finished
 constexpr int kDkCtrItems = 3;      // items handed out beyond the first gridDim.x
-constexpr int kDkCtrUnits = 4;      // conversion units handed out
-constexpr int kDkCtrUnitsDone = 5;  // conversion units written
+constexpr int kDkCtrUnitsDone = 5;  // CTAs whose conversion units are all written
 
 // Bytes of converted B operands of one stage of a layer with M tokens: the
-// integer engine needs 8 KB per column group (2 groups at M = 2), the fp16
-// engine 1 KB per token and segment (tokens rounded up to even).
+// integer engine needs 4 KB per column group (2 groups at M = 2), the fp16
+// engine 1 KB per token (tokens rounded up to even).
 __host__ __device__ constexpr uint32_t dk_stage_b(int M) {
-    return M <= 1 ? 8192u : (M == 2 ? 16384u : 2048u * (uint32_t)(M + (M & 1)));
+    return M <= 1 ? 4096u : (M == 2 ? 8192u : 1024u * (uint32_t)(M + (M & 1)));
 }
 // Consumer -> epilogue buffer: [token][warp][tile][row] of int64 (M <= 2) or fp32.
 __host__ __device__ constexpr uint32_t dk_part_bytes(int maxM) {
@@ -175,37 +173,37 @@ struct DkArgs {
     int total_items;
     int total_units;
     int maxM;
-    int chained;  // some layer converts per item (raw activation buffers needed)
+    int chained;  // some layer reads an earlier layer's output
 };
 
 struct DkQEntry {
     uint16_t *Y;
+    const uint16_t *X;
     int64_t part_off;
     float alpha;
     int item;  // -1: no more items
-    int tile, part, s0, s1, M, K, N, ldy, parts, tile_begin, pre;
-    int pad_;
+    int tile, part, s0, s1, M, K, N, ldx, ldy, parts, tile_begin;
+    int pre;   // 1: converted operands arrive with the weights; 0: a stager converts X
 };
 
 struct DkLayout {
-    uint32_t ns, raw_stage, slot_b, parts, w_off, raw_off, st_off, part_off, q_off, bar_off, total;
-    __host__ __device__ DkLayout(int maxM, int chained) {
-        raw_stage = chained ? (uint32_t)kDkRawTok * (uint32_t)maxM : 0u;
-        slot_b = (maxM <= 1 ? 8192u : 16384u) + kDkMetaBytes;  // [meta][B]
+    uint32_t ns, nbufs, slot_b, parts, w_off, st_off, part_off, q_off, bar_off, total;
+    __host__ __device__ explicit DkLayout(int maxM) {
+        slot_b = (maxM <= 1 ? 4096u : 8192u) + kDkMetaBytes;  // [meta][B]
         parts = dk_part_bytes(maxM);
-        const uint32_t per_stage = (uint32_t)kDkWBytes + raw_stage + slot_b;
-        const uint32_t fixed = kDkPartBufs * parts + kDkQueue * (uint32_t)sizeof(DkQEntry) +
-                               8u * (3u * kDkMaxStages + 2u * kDkQueue + 2u * kDkPartBufs) +
-                               1024u;  // alignment slack of the dynamic base
+        nbufs = parts <= 8192u ? (uint32_t)kDkMaxPartBufs : 2u;
+        const uint32_t per_stage = (uint32_t)kDkWBytes + slot_b;
+        const uint32_t fixed = nbufs * parts + kDkQueue * (uint32_t)sizeof(DkQEntry) +
+                               8u * (3u * kDkMaxStages + 2u * kDkQueue + 2u * kDkMaxPartBufs) +
+                               16u + 1024u;  // a counter; alignment slack of the dynamic base
         const uint32_t n = (kDkSmemBudget - fixed) / per_stage;
         ns = n > (uint32_t)kDkMaxStages ? (uint32_t)kDkMaxStages : n;  // >= 3 for maxM <= 8
         w_off = 0;
-        raw_off = ns * (uint32_t)kDkWBytes;
-        st_off = raw_off + ns * raw_stage;
+        st_off = ns * (uint32_t)kDkWBytes;
         part_off = st_off + ns * slot_b;
-        q_off = part_off + kDkPartBufs * parts;
+        q_off = part_off + nbufs * parts;
         bar_off = (q_off + kDkQueue * (uint32_t)sizeof(DkQEntry) + 7u) & ~7u;
-        total = bar_off + 8u * (3u * ns + 2u * kDkQueue + 2u * kDkPartBufs) + 1024u;
+        total = bar_off + 8u * (3u * ns + 2u * kDkQueue + 2u * nbufs) + 16u + 1024u;
     }
 };
 
@@ -306,19 +304,19 @@ __host__ __device__ constexpr int dk_col(int m, int p) { return 6 * m + p; }
 __host__ __device__ constexpr int dk_ones_col(int M) { return 6 * M; }
 
 // Offset of the 16-byte B block of (16-trit word w of the stage, column col)
-// in the integer engine's layout: [cg][segment][v][i][col & 7][c], where
-// w = segment * 32 + (4 v + c) * 4 + i.  A consumer quarter-warp reads two
-// columns x four c: 128 contiguous bytes.
+// in the integer engine's layout: [cg][v][i][col & 7][c], where
+// w = (4 v + c) * 4 + i.  A consumer quarter-warp reads two columns x four c:
+// 128 contiguous bytes.
 __device__ __forceinline__ uint32_t dk_iblock(int w, int col) {
-    const int h = w >> 5, ch = (w >> 2) & 7, i = w & 3, v = ch >> 2, c = ch & 3;
-    return (uint32_t)((col >> 3) * 8192 + h * 4096 + (((v * 4 + i) * 8 + (col & 7)) * 4 + c) * 16);
+    const int ch = w >> 2, i = w & 3, v = ch >> 2, c = ch & 3;
+    return (uint32_t)((col >> 3) * 4096 + (((v * 4 + i) * 8 + (col & 7)) * 4 + c) * 16);
 }
 // fp16 engine: offset of the 16-byte half `hf` (digit positions 2hf, 2hf+1)
-// of the B operands of (word w, token m): [segment][v][i][hf][m][c], Mp =
-// tokens rounded up to even (a quarter-warp reads tokens 2p, 2p+1 x four c).
+// of the B operands of (word w, token m): [v][i][hf][m][c], Mp = tokens rounded
+// up to even (a quarter-warp reads tokens 2p, 2p+1 x four c).
 __device__ __forceinline__ uint32_t dk_hblock(int w, int m, int hf, int Mp) {
-    const int h = w >> 5, ch = (w >> 2) & 7, i = w & 3, v = ch >> 2, c = ch & 3;
-    return (uint32_t)(h * 1024 * Mp + ((((v * 4 + i) * 2 + hf) * Mp + m) * 4 + c) * 16);
+    const int ch = w >> 2, i = w & 3, v = ch >> 2, c = ch & 3;
+    return (uint32_t)(((((v * 4 + i) * 2 + hf) * Mp + m) * 4 + c) * 16);
 }
 
 // MMA row g of a 16-row tile reads physical row pi(g) (and pi(g) + 8).
@@ -357,7 +355,7 @@ __device__ __forceinline__ void dk_conv_imma(const uint16_t *src, int valid, int
                                              uint8_t *dstB, uint8_t *meta, int lane) {
     const int ones = dk_ones_col(M);
     double qd = 0.0;
-    for (int w = lane; w < 64; w += 32) {
+    for (int w = lane; w < kDkWords; w += 32) {
         uint32_t r[8];
         dk_read_word(src, w, valid, r);
         uint32_t lo[16], hi[16];
@@ -408,7 +406,7 @@ __device__ __forceinline__ void dk_conv_imma(const uint16_t *src, int valid, int
 __device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, int valid, int m, int Mp,
                                              uint8_t *dstB, uint8_t *meta, int lane) {
     float sx = 0.f;
-    for (int w = lane; w < 64; w += 32) {
+    for (int w = lane; w < kDkWords; w += 32) {
         uint32_t r[8];
         dk_read_word(src, w, valid, r);
         uint32_t b[8];
@@ -433,22 +431,23 @@ __device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, int valid, int
 
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
     extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
-    const DkLayout lay(a.maxM, a.chained);
+    const DkLayout lay(a.maxM);
     const int NS = (int)lay.ns;
     // 1024-byte alignment for the 128-byte swizzle of the weight boxes
     uint8_t *smem = dk_smem_raw + ((1024u - (smem_u32(dk_smem_raw) & 1023u)) & 1023u);
     uint8_t *wring = smem + lay.w_off;
-    uint8_t *rawx = smem + lay.raw_off;
     uint8_t *sslot = smem + lay.st_off;  // per slot: [meta 64 B][B operands]
     uint8_t *parts = smem + lay.part_off;
     DkQEntry *queue = reinterpret_cast<DkQEntry *>(smem + lay.q_off);
     uint64_t *wfull = reinterpret_cast<uint64_t *>(smem + lay.bar_off);  // copies landed
-    uint64_t *xfull = wfull + NS;                                         // stager -> consumers
+    uint64_t *xfull = wfull + NS;  // stager -> consumers (stages converted on chip only)
     uint64_t *empty = xfull + NS;                                         // consumers -> producer
     uint64_t *qfull = empty + NS;
     uint64_t *qempty = qfull + kDkQueue;
+    const int NB = (int)lay.nbufs;
     uint64_t *pfull = qempty + kDkQueue;  // consumers -> epilogue
-    uint64_t *pempty = pfull + kDkPartBufs;
+    uint64_t *pempty = pfull + NB;
+    uint32_t *conv_done = reinterpret_cast<uint32_t *>(pempty + NB);  // warps done converting
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -461,10 +460,11 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             mbar_init(&qfull[i], 1);
             mbar_init(&qempty[i], kDkConsumers + kDkStagers + kDkEpilogues);
         }
-        for (int i = 0; i < kDkPartBufs; ++i) {
+        for (int i = 0; i < NB; ++i) {
             mbar_init(&pfull[i], kDkConsumers);
             mbar_init(&pempty[i], 1);
         }
+        *conv_done = 0u;
         fence_mbar_init();
     }
     __syncthreads();
@@ -473,11 +473,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
     if (warp != 0) {
         // ---- every warp but the producer: convert activations, one unit at a time ----
         pdl_wait();  // X may be written by the preceding grid; Y may still be in use
-        while (true) {
-            int u = 0;
-            if (lane == 0) u = (int)atomicAdd(&a.ctr[kDkCtrUnits], 1u);
-            u = __shfl_sync(0xffffffffu, u, 0);
-            if (u >= a.total_units) break;
+        // unit u goes to warp u mod (all converting warps of the grid)
+        constexpr int kConv = kDkWarps - 1;
+        for (int u = (int)blockIdx.x * kConv + warp - 1; u < a.total_units;
+             u += (int)gridDim.x * kConv) {
             const DkUnitRec U = dk_load_rec<DkUnitRec, 3>(a.units, u);
             const int valid = min(U.K - U.stage * kDkStageTrits, kDkStageTrits);
             const uint16_t *src = U.X + (int64_t)U.m * U.ldx + (int64_t)U.stage * kDkStageTrits;
@@ -489,10 +488,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             dk_fence_proxy_global();
             __threadfence();
             __syncwarp();
-            if (lane == 0) {
-                atomicAdd(&a.ready[U.layer], 1u);
-                atomicAdd(&a.ctr[kDkCtrUnitsDone], 1u);
-            }
+            if (lane == 0) atomicAdd(&a.ready[U.layer], 1u);
+        }
+        // the last converting warp of the CTA counts the CTA as done
+        if (lane == 0 && atomicAdd(conv_done, 1u) == (uint32_t)kConv - 1) {
+            __threadfence();
+            atomicAdd(&a.ctr[kDkCtrUnitsDone], 1u);
         }
     }
 
@@ -507,7 +508,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         uint32_t pph = 0;
         bool wrapped = false;
         int qi = 0;
-        bool waited = false, ok = true, all_ready = a.total_units == 0;
+        bool waited = false, ok = true, all_ready = a.total_units == 0, fenced = true;
         uint32_t final_seen = 0;
         const int G = (int)gridDim.x;
         int item = (int)blockIdx.x;
@@ -527,6 +528,8 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 e.item = valid ? item : -1;
                 if (valid) {
                     e.Y = R.Y;
+                    e.X = R.X;
+                    e.ldx = R.ldx;
                     e.part_off = R.part_off;
                     e.alpha = R.alpha;
                     e.tile = R.tile;
@@ -548,48 +551,37 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             if (!valid) break;
             const CUtensorMap *tmap = a.maps + R.layer;
             const int n0 = R.tile * kDkRows;
-            // activation bytes of stage s for one token (whole 16-byte units)
-            auto xbytes = [&](int s) -> uint32_t {
-                const int rem = R.K - s * kDkStageTrits;
-                const int n = rem < kDkStageTrits ? ((rem + 7) & ~7) : kDkStageTrits;
-                return 2u * (uint32_t)n;
-            };
-            // bytes of a stage besides the weights
-            auto extra = [&](int s) -> uint32_t {
-                return pre ? (uint32_t)R.bstride : (uint32_t)R.M * xbytes(s);
-            };
+            // bytes of a stage besides the weights: the converted operands
+            auto extra = [&](int) -> uint32_t { return pre ? (uint32_t)R.bstride : 0u; };
             auto issue_w = [&](int slot, int s) {
                 tma_load_2d(wring + slot * kDkWBytes, tmap, &wfull[slot], s * kDkStageW, n0);
-                tma_load_2d(wring + slot * kDkWBytes + kDkBoxBytes, tmap, &wfull[slot],
-                            s * kDkStageW + kDkSegBytes, n0);
             };
             auto issue_x = [&](int slot, int s) {
-                if (pre) {
+                if (pre)
                     dk_bulk_load(sslot + slot * lay.slot_b, R.B + (int64_t)s * R.bstride,
                                  (uint32_t)R.bstride, &wfull[slot]);
-                } else {
-                    const uint32_t b = xbytes(s);
-                    for (int m = 0; m < R.M; ++m)
-                        dk_bulk_load(rawx + slot * lay.raw_stage + m * kDkRawTok,
-                                     R.X + (int64_t)m * R.ldx + (int64_t)s * kDkStageTrits, b,
-                                     &wfull[slot]);
-                }
             };
             // the item's activations may be read: the layer's units are
             // converted, or (chained layers) the earlier layers' outputs are final
             auto wait_inputs = [&]() -> bool {
                 bool good = true;
                 if (pre) {
-                    if (!all_ready)
+                    if (!all_ready) {
                         good = dk_wait_count(&a.ready[R.layer], (uint32_t)R.need,
-                                             &a.ctr[kDkCtrUnitsDone], (uint32_t)a.total_units,
-                                             &all_ready);
+                                             &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
+                        fenced = false;
+                    }
                 } else if (R.wait_tiles > 0 && final_seen < (uint32_t)R.wait_tiles) {
                     good = dk_wait_count(&a.ctr[kDkCtrFinal], (uint32_t)R.wait_tiles, nullptr, 0u,
                                          nullptr);
                     if (good) final_seen = (uint32_t)R.wait_tiles;
+                    fenced = false;
                 }
-                dk_fence_proxy_global();
+                // what was observed above is read next by bulk copies (async proxy)
+                if (!fenced) {
+                    dk_fence_proxy_global();
+                    fenced = true;
+                }
                 return good;
             };
             int s = R.s0;
@@ -673,10 +665,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             mbar_wait(&wfull[t % NS], (t / NS) & 1u);
     } else if (warp < kDkFirstEpi) {
         // ---------------- stagers ----------------
-        // Converted stages only need their arrival; per-item stages (chained
-        // layers) are converted here from the raw activations.  Either way the
-        // stager first waits for the stage's copies, so xfull never runs a
-        // round ahead of the consumers.
+        // Stages whose operands were converted beforehand pass them by; the
+        // others (chained layers) are converted here from X
+        // in global memory once the stage's weights have landed -- after the
+        // producer's wait for the inputs, so X is final.  A stage's weights
+        // arriving also means the consumers have released the slot's previous
+        // round, so xfull is never arrived on a round ahead.
         const int sw = warp - 1;
         int ss = 0;
         uint32_t sph = 0;
@@ -692,44 +686,46 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     ss = 0;
                     sph ^= 1u;
                 }
-                if (slot % kDkStagers != sw) continue;  // another stager's slot
+                if (e.pre || slot % kDkStagers != sw) continue;  // converted, or another stager's
                 if (!dk_warp_wait(&wfull[slot], ph)) {
                     ok = false;
                     break;
                 }
-                if (!e.pre) {
-                    const int valid = min(K - s * kDkStageTrits, kDkStageTrits);
-                    uint8_t *dst = sslot + slot * lay.slot_b;
-                    for (int m = 0; m < M; ++m) {
-                        const uint16_t *src = reinterpret_cast<const uint16_t *>(
-                            rawx + slot * lay.raw_stage + m * kDkRawTok);
-                        if (M <= kDkImmaMaxM)
-                            dk_conv_imma(src, valid, m, M, dst + kDkMetaBytes, dst, lane);
-                        else
-                            dk_conv_hmma(src, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
-                    }
+                const int valid = min(K - s * kDkStageTrits, kDkStageTrits);
+                uint8_t *dst = sslot + slot * lay.slot_b;
+                for (int m = 0; m < M; ++m) {
+                    const uint16_t *src = e.X + (int64_t)m * e.ldx + (int64_t)s * kDkStageTrits;
+                    if (M <= kDkImmaMaxM)
+                        dk_conv_imma(src, valid, m, M, dst + kDkMetaBytes, dst, lane);
+                    else
+                        dk_conv_hmma(src, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
                 }
                 mbar_arrive(&xfull[slot]);
             }
         }
     } else if (warp < kDkFirstCons) {
-        // ---------------- epilogues: warp 4 + i takes the items i, i + 2, ... ----------------
+        // ---------------- epilogues ----------------
+        // Item i uses buffer i mod NB and goes to epilogue warp i mod EA, with
+        // EA = min(warps, NB) dividing NB: each warp owns its buffers and waits
+        // on their phases in order (a parity wait must never be a phase ahead).
         const int ew = warp - kDkFirstEpi;
+        const int EA = NB < kDkEpilogues ? NB : kDkEpilogues;
         int qi = 0, pi = -1;
         DkQEntry e;
         while (dk_next_item(queue, qfull, qempty, qi, e)) {
-            if (++pi % kDkEpilogues != ew) continue;
-            const int b = pi % kDkPartBufs;
-            if (!dk_warp_wait(&pfull[b], (uint32_t)(pi / kDkPartBufs) & 1u)) break;
+            if (++pi % EA != ew) continue;
+            const int b = pi % NB;
+            if (!dk_warp_wait(&pfull[b], (uint32_t)(pi / NB) & 1u)) break;
             const uint8_t *pb = parts + b * lay.parts;
             const int M = e.M, n0 = e.tile * kDkRows, cnt = kDkRows * M;
             const bool exact = M <= kDkImmaMaxM;
             int64_t *slot = e.parts > 1 ? a.partials + e.part_off +
                                               (int64_t)(e.tile * e.parts + e.part) * cnt
                                         : nullptr;
-            // partial of (token m, warp cw, tile t, MMA row rho) at ((m*16 + cw)*2 + t)*16 + rho;
-            // the four warps of a row tile (cw, cw + 4, +8, +12) are 128 entries
-            // apart, and 32 consecutive rows of one token read 32 consecutive entries
+            // partial of (token m, warp cw, tile pair tile t, MMA row rho) at
+            // ((m*16 + cw)*2 + t)*16 + rho; the two warps of a row tile (cw, cw + 8)
+            // are 256 entries apart, and 32 consecutive rows of one token read 32
+            // consecutive entries
             for (int idx = lane; idx < cnt; idx += 32) {
                 const int r = idx % kDkRows, m = idx / kDkRows;  // consecutive lanes: consecutive n
                 const int t = r >> 4, tp = t >> 1, tl = t & 1;
@@ -737,7 +733,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 const int base = ((m * 16 + tp) * 2 + tl) * 16 + rho;
                 if (exact) {
                     const int64_t *p = reinterpret_cast<const int64_t *>(pb);
-                    const int64_t v = p[base] + p[base + 128] + p[base + 256] + p[base + 384];
+                    const int64_t v = p[base] + p[base + 256];
                     if (slot) {
                         slot[idx] = v;
                     } else if (n0 + r < e.N) {
@@ -746,7 +742,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                 } else {
                     const float *p = reinterpret_cast<const float *>(pb);
-                    const float v = ((p[base] + p[base + 128]) + p[base + 256]) + p[base + 384];
+                    const float v = p[base] + p[base + 256];
                     if (slot) {
                         reinterpret_cast<double *>(slot)[idx] = (double)v;
                     } else if (n0 + r < e.N) {
@@ -824,22 +820,26 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
     } else {
         // ---------------- consumers ----------------
         const int cw = warp - kDkFirstCons;
-        const int tp = cw & 3, qv = cw >> 2;
-        const int h = qv >> 1, v = qv & 1;
+        const int tp = cw & 7, v = cw >> 3;  // tile pair, half of the stage's 128 bytes
+        const int qv = v;                     // the warp that subtracts the offsets: v == 0
         const int g = lane >> 2, c = lane & 3;
         const int pg = dk_pi(g);
         // tile 2tp, MMA row g: physical row 32 tp + pg; the 4 rows of this lane
         // (tiles 2tp / 2tp+1, rows g / g+8) are 8 rows apart
-        const uint32_t aoff = (uint32_t)((32 * tp + pg) * kDkSegBytes + (((4 * v + c) ^ pg) << 4)) +
-                              (uint32_t)h * kDkBoxBytes;
+        const uint32_t aoff = (uint32_t)((32 * tp + pg) * kDkStageW + (((4 * v + c) ^ pg) << 4));
         int cs = 0;
         uint32_t cph = 0;
+        uint32_t xph = 0;  // bit s: parity of slot s's next xfull phase
         int qi = 0, pi = 0;
         bool ok = true;
-        DkQEntry e;
-        // waits for the stage's copies and conversion; false on a timeout
+        DkQEntry e{};
+        // waits for the stage's copies (and its conversion on chip); false on a timeout
         auto wait_stage = [&](int slot) -> bool {
-            return dk_warp_wait(&wfull[slot], cph) && dk_warp_wait(&xfull[slot], cph);
+            if (!dk_warp_wait(&wfull[slot], cph)) return false;
+            if (e.pre) return true;
+            const bool good = dk_warp_wait(&xfull[slot], (xph >> slot) & 1u);
+            xph ^= 1u << slot;
+            return good;
         };
         auto release = [&](int slot) {
             // the shared-memory values are consumed (in registers) before the release
@@ -852,7 +852,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         };
         while (ok && dk_next_item(queue, qfull, qempty, qi, e)) {
             const int M = e.M;
-            const int b = pi % kDkPartBufs;
+            const int b = pi % NB;
             uint8_t *pb = parts + b * lay.parts;
             if (M == 1) {
                 // ---- integer engine, one token: one accumulator per digit
@@ -871,12 +871,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                     const uint8_t *wb = wring + slot * kDkWBytes + aoff;
                     const uint4 A00 = dk_lds128(wb);                     // tile 2tp, row g
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);   // tile 2tp, row g + 8
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);  // tile 2tp + 1, row g
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);  // tile 2tp + 1, row g + 8
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);   // tile 2tp, row g + 8
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);  // tile 2tp + 1, row g
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);  // tile 2tp + 1, row g + 8
                     const uint8_t *sb = sslot + slot * lay.slot_b;
                     qsum += reinterpret_cast<const int64_t *>(sb)[0];
-                    const uint8_t *xg = sb + kDkMetaBytes + h * 4096 + ((v * 32 + g) * 4 + c) * 16;
+                    const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
 #pragma unroll
                     for (int pr = 0; pr < 2; ++pr) {
                         const int i0 = 2 * pr, i1 = i0 + 1;
@@ -894,27 +894,36 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     release(slot);
                 }
                 if (!ok) break;
-                if (pi >= kDkPartBufs &&
-                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
                     break;
                 // V = sum_p 256^p S_p - 2^40 S_ones - Q; this lane holds columns
                 // 2c, 2c + 1 (planes 2c, 2c + 1, or the ones column at c = 3)
+                // D = 64 S exactly: position j carries 4^j, so acc0*64 + acc1*16 +
+                // acc2*4 + acc3 = 64 sum_j acc_j 4^-j (below 2^31 for items of at most
+                // kDkMaxItemStages stages); lane c's columns give t_c = D_2c + 256 D_2c+1
+                // (lane 3: the ones column), and lane 0 forms
+                // 64 V = t_0 + 2^16 t_1 + 2^32 t_2 - 2^40 t_3 - 64 Q (modulo 2^64).
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
 #pragma unroll
                     for (int rr = 0; rr < 2; ++rr) {
-                        int64_t d[2];
+                        uint32_t d[2];
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
-                            const int q = 2 * rr + u;  // digit positions carry 4^j, exactly divisible
-                            d[u] = (int64_t)(acc[t][0][q] + (acc[t][1][q] >> 2) + (acc[t][2][q] >> 4) +
-                                             (acc[t][3][q] >> 6));
+                            const int q = 2 * rr + u;
+                            d[u] = (uint32_t)(acc[t][0][q] * 64 + acc[t][1][q] * 16 + acc[t][2][q] * 4 +
+                                              acc[t][3][q]);
                         }
-                        int64_t v0 = c < 3 ? (d[0] << (16 * c)) + (d[1] << (16 * c + 8)) : -(d[0] << 40);
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-                        if (qv == 0) v0 -= qsum;
-                        if (c == 0) reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                        const uint64_t tc = c < 3 ? (uint64_t)d[0] + ((uint64_t)d[1] << 8) : (uint64_t)d[0];
+                        const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
+                        const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
+                        const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
+                        if (c == 0) {
+                            uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 40);
+                            if (qv == 0) v64 -= (uint64_t)qsum << 6;
+                            reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] =
+                                (int64_t)v64 >> 6;
+                        }
                     }
                 }
             } else if (M == 2) {
@@ -934,19 +943,19 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                     const uint8_t *wb = wring + slot * kDkWBytes + aoff;
                     const uint4 A00 = dk_lds128(wb);
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
                     const uint8_t *sb = sslot + slot * lay.slot_b;
                     qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
                     qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
-                    const uint8_t *xg = sb + kDkMetaBytes + h * 4096 + ((v * 32 + g) * 4 + c) * 16;
+                    const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
 #pragma unroll
                     for (int pr = 0; pr < 2; ++pr) {
                         const int i0 = 2 * pr, i1 = i0 + 1;
                         const uint4 B00 = dk_lds128(xg + i0 * 512), B01 = dk_lds128(xg + i1 * 512);
-                        const uint4 B10 = dk_lds128(xg + 8192 + i0 * 512);
-                        const uint4 B11 = dk_lds128(xg + 8192 + i1 * 512);
+                        const uint4 B10 = dk_lds128(xg + 4096 + i0 * 512);
+                        const uint4 B11 = dk_lds128(xg + 4096 + i1 * 512);
 #pragma unroll 2
                         for (int j = 0; j < 4; ++j) {
                             constexpr uint32_t m = 0x03030303u;
@@ -969,8 +978,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     release(slot);
                 }
                 if (!ok) break;
-                if (pi >= kDkPartBufs &&
-                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
                     break;
                 // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
                 // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
@@ -1022,9 +1030,9 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                     const uint8_t *wb = wring + slot * kDkWBytes + aoff;
                     const uint4 A00 = dk_lds128(wb);
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkSegBytes);
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkSegBytes);
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkSegBytes);
+                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
+                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
+                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
                     const uint8_t *sb = sslot + slot * lay.slot_b;
                     const float *mt = reinterpret_cast<const float *>(sb);
                     if (2 * c < M) sx0 += mt[2 * c];
@@ -1034,7 +1042,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     for (int i = 0; i < 4; ++i) {
                         uint4 B0 = make_uint4(0u, 0u, 0u, 0u), B1 = B0;
                         if (g < M) {
-                            const int w = h * 32 + (4 * v + c) * 4 + i;
+                            const int w = (4 * v + c) * 4 + i;
                             B0 = dk_lds128(xb + dk_hblock(w, g, 0, Mp));
                             B1 = dk_lds128(xb + dk_hblock(w, g, 1, Mp));
                         }
@@ -1054,8 +1062,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     release(slot);
                 }
                 if (!ok) break;
-                if (pi >= kDkPartBufs &&
-                    !dk_warp_wait(&pempty[b], (uint32_t)((pi / kDkPartBufs) - 1) & 1u))
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
                     break;
                 float *p = reinterpret_cast<float *>(pb);
 #pragma unroll
@@ -1097,7 +1104,6 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             __threadfence();
             a.ctr[kDkCtrFinal] = 0u;
             a.ctr[kDkCtrItems] = 0u;
-            a.ctr[kDkCtrUnits] = 0u;
             a.ctr[kDkCtrUnitsDone] = 0u;
             for (int l = 0; l < a.count; ++l) a.ready[l] = 0u;
             a.ctr[kDkCtrDone] = 0u;
@@ -1110,10 +1116,18 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
 // ---- host side ---------------------------------------------------------------
 namespace tlk {
 
-// K-parts of a layer: items of about kDkItemStages stages, cut at stage
+// Stages per item for a batch of `total` stages: about six items per SM of a
+// B200, so the last items leave little tail, but between 8 and 16 stages
+// (4096 to 8192 trits of K), so item boundaries (and the epilogue work per
+// item) stay rare.
+inline int dk_item_stages(int64_t total) {
+    const int64_t t = total / (6 * kDkRefSms);
+    return t < 8 ? 8 : (t > 16 ? 16 : (int)t);
+}
+// K-parts of a layer: items of about `target` stages, cut at stage
 // boundaries, never more than kDkMaxItemStages stages per item.
-inline int dk_parts(int stages) {
-    int parts = (stages + kDkItemStages / 2) / kDkItemStages;
+inline int dk_parts(int stages, int target) {
+    int parts = (stages + target / 2) / target;
     if (parts < 1) parts = 1;
     while ((stages + parts - 1) / parts > kDkMaxItemStages) ++parts;
     if (parts > stages) parts = stages;
@@ -1138,15 +1152,23 @@ struct DkSchedule {
 
 // Sizes of a batch; with `items` and `units` given, also their tables, holding
 // pointers into the workspace at `ws`.  Items are in layer order, then tile,
-// then part; units in layer order, then stage, then token.
+// then part (longest first when no layer reads an earlier one); units in
+// layer order, then stage, then token.
 inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
                               std::vector<DkItemRec> *items, std::vector<DkUnitRec> *units) {
     DkSchedule sc;
     sc.count = count;
+    auto stages_of = [](const DkHostLayer &h) {
+        return (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
+    };
+    int64_t total = 0;
+    for (int l = 0; l < count; ++l)
+        total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows);
+    const int target = dk_item_stages(total);
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
-        const int stages = (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
-        const int parts = dk_parts(stages);
+        const int stages = stages_of(h);
+        const int parts = dk_parts(stages, target);
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         sc.total_items += tiles * parts;
         sc.total_tiles += tiles;
@@ -1166,8 +1188,8 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     int tile_begin = 0;
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
-        const int stages = (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
-        const int parts = dk_parts(stages);
+        const int stages = stages_of(h);
+        const int parts = dk_parts(stages, target);
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         const int bstride = kDkMetaBytes + (int)dk_stage_b(h.M);
         uint8_t *B = h.reads_earlier ? nullptr : ws + wl.staged + staged;
@@ -1214,18 +1236,25 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         if (B) staged += (int64_t)stages * bstride;
         tile_begin += tiles;
     }
+    // Items are handed out in table order.  Without dependencies between
+    // layers, the longest items go first, so the last ones handed out (the
+    // launch's tail) are the shortest.
+    if (!sc.chained)
+        std::stable_sort(items->begin(), items->end(), [](const DkItemRec &x, const DkItemRec &y) {
+            return x.s1 - x.s0 > y.s1 - y.s0;
+        });
     return sc;
 }
 
 // Tensor map of a layer's packed weights: bytes x rows, boxes of 128 bytes x
-// 128 rows with the 128-byte swizzle, zero fill outside [0, row bytes) x [0, N).
+// 256 rows with the 128-byte swizzle, zero fill outside [0, row bytes) x [0, N).
 inline bool dk_encode_map(const DkHostLayer &h, CUtensorMap *map) {
     auto encode = tensor_map_encoder();
     if (!encode) return false;
     const int64_t rowbytes = ((int64_t)h.K + 3) / 4;
     cuuint64_t dims[2] = {(cuuint64_t)rowbytes, (cuuint64_t)h.N};
     cuuint64_t strides[1] = {(cuuint64_t)h.ldp};
-    cuuint32_t box[2] = {(cuuint32_t)kDkSegBytes, (cuuint32_t)kDkRows};
+    cuuint32_t box[2] = {(cuuint32_t)kDkStageW, (cuuint32_t)kDkRows};
     cuuint32_t estr[2] = {1, 1};
     return encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(h.T), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -1267,7 +1296,7 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     std::call_once(once[dev], [dev] {
         uint32_t most = 0;
         for (int m = 1; m <= 8; ++m) {
-            const uint32_t t = DkLayout(m, 1).total;
+            const uint32_t t = DkLayout(m).total;
             most = t > most ? t : most;
         }
         attr_err[dev] = cudaFuncSetAttribute(decode2_kernel,
@@ -1280,7 +1309,7 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.total_items < num_sms ? a.total_items : num_sms));
     cfg.blockDim = dim3(kDkThreads);
-    cfg.dynamicSmemBytes = DkLayout(a.maxM, a.chained).total;
+    cfg.dynamicSmemBytes = DkLayout(a.maxM).total;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -111,23 +111,26 @@ def _up(v):
 def _ws2_expected(layers):
     """2-bit batch workspace, region by region (each rounded up to 256 bytes):
     counters, one 128-byte tensor map per layer, a 96-byte record per work item
-    (128-row tile x K-part), a 48-byte record per conversion unit (stage x token
-    of a layer that reads no earlier output), a u32 per layer and per tile,
-    8-byte partials of split tiles, and the converted activations
-    (64 + 8 KB, 16 KB or 2 KB x even(M) bytes per stage)."""
+    (256-row tile x K-part of 8..16 stages of 512 trits), a 48-byte record per
+    conversion unit (stage x token of a layer that reads no earlier output), a
+    u32 per layer and per tile, 8-byte partials of split tiles, and the
+    converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage)."""
     items = units = tiles = slots = staged = 0
+    stg = lambda d: -(-(-(-d["K"] // 4)) // 128)
+    total = sum(stg(d) * -(-d["N"] // 256) for d in layers)
+    target = min(16, max(8, total // (6 * 148)))  # stages per item
     for d in layers:
-        stages = -(-(-(-d["K"] // 4)) // 256)
-        parts = max(1, min(stages, (stages + 2) // 4))
-        t = -(-d["N"] // 128)
+        stages = stg(d)
+        parts = max(1, min(stages, (stages + target // 2) // target))
+        t = -(-d["N"] // 256)
         items += t * parts
         tiles += t
         if not d.get("flags", 0):
             units += stages * d["M"]
-            b = 8192 if d["M"] == 1 else (16384 if d["M"] == 2 else 2048 * (d["M"] + d["M"] % 2))
+            b = 4096 if d["M"] == 1 else (8192 if d["M"] == 2 else 1024 * (d["M"] + d["M"] % 2))
             staged += stages * (64 + b)
         if parts > 1:
-            slots += t * parts * 128 * d["M"]
+            slots += t * parts * 256 * d["M"]
     off = 256
     for size in (128 * len(layers), 96 * items, 48 * units, 4 * len(layers), 4 * tiles, 8 * slots,
                  staged):
@@ -139,7 +142,8 @@ def test_batch_workspace_size(L):
     base = dict(M=1, flags=0)
     cases = [[dict(base, N=1000, K=2048)], [dict(base, N=4096, K=14336)],
              [dict(base, N=4096, K=14336, M=8)], [dict(base, N=4096, K=14336, M=2)],
-             [dict(base, N=130, K=700, M=3), dict(base, N=77, K=5000, M=1, flags=1)]]
+             [dict(base, N=130, K=700, M=3), dict(base, N=77, K=5000, M=1, flags=1)],
+             [dict(base, N=14336, K=4096)] * 12, [dict(base, N=3072, K=8192, M=8)] * 80]
     for ls in cases:
         arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16, ldx=d["K"] +
                             (-d["K"]) % 8, ldy=d["N"] + (-d["N"]) % 8) for d in ls])
