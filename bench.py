@@ -154,11 +154,17 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # inputs
 # ---------------------------------------------------------------------------
-def make_matrix(fmt: int, K: int, N: int, seed: int, p0: float = 1.0 / 3.0):
-    """Packed weights (product codec), trits and alpha of one seeded matrix."""
+def make_matrix(fmt: int, K: int, N: int, seed: int, p0: float = 1.0 / 3.0,
+                codec: str = "product"):
+    """Packed weights, trits and alpha of one seeded matrix.  codec="product"
+    packs with the library (the GPU arm's inputs); codec="oracle" with the
+    CPU oracle's own packer (the CPU arms, which load nothing of the library)."""
     import synth
-    import ternary_weight_03_b200 as tl
     T = synth.trits(seed, N, K, p0=p0)
+    if codec == "oracle":
+        import oracle
+        return oracle.get().pack(fmt, T), T, synth.alpha_for(seed)
+    import ternary_weight_03_b200 as tl
     return tl.pack(fmt, T), T, synth.alpha_for(seed)
 
 
@@ -246,30 +252,43 @@ class Sweep:
                     events[j].record(stream)
 
 
+# steps per CUDA graph in the timed region: consecutive launches inside one
+# graph are chained by programmatic dependent launch (a launch streams its
+# first weights while its predecessor drains); between graph replays they are not
+GRAPH_STEPS = 45
+
+
 def time_graphs(sweep: Sweep, steps: int, warmup: int, stream, clock_gpu: int | None = None,
                 flags: int = 1):
-    """Capture one CUDA graph per rotation phase, warm up, then time `steps`
-    replays with CUDA events on the launch stream.  The timed graphs hold the
-    layer calls only (event nodes between them would cut the programmatic
-    dependent-launch edges).  Afterwards one untimed replay of graphs with
-    event records between the calls, launched without PDL, gives a per-call
-    breakdown.  Returns (total ms, per-call ms list, clocks summary)."""
+    """Warm up with `warmup` steps, then time exactly `steps` steps with CUDA
+    events on the launch stream.  Steps are captured into CUDA graphs of up to
+    GRAPH_STEPS consecutive steps (the rotation phases advance from step to
+    step), so the timed region replays steps // GRAPH_STEPS such graphs and one
+    graph of the remaining steps.  The timed graphs hold the layer calls only.
+    Afterwards one untimed replay of graphs with event records between the
+    calls, launched without PDL, gives a per-call breakdown.  Returns (total
+    ms, per-call ms list, clocks summary)."""
     import torch
     nm = len(sweep.ms)
     nphase = sweep.copies // nm if sweep.copies % nm == 0 else sweep.copies
     if sweep.batch:
         nphase = len(sweep.plans)
-    graphs = []
+
+    def capture(first, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                sweep.enqueue((first + i) % nphase, stream, flags=flags)
+        return g
+
     with torch.cuda.stream(stream):
         sweep.enqueue(0, stream, flags=flags)  # per-device setup outside capture
         torch.cuda.synchronize()
-        for ph in range(nphase):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                sweep.enqueue(ph, stream, flags=flags)
-            graphs.append(g)
-        for s in range(warmup):
-            graphs[s % nphase].replay()
+        g_warm = capture(0, warmup)
+        full, rem = divmod(steps, GRAPH_STEPS)
+        g_full = capture(warmup % nphase, GRAPH_STEPS) if full else None
+        g_rem = capture((warmup + full * GRAPH_STEPS) % nphase, rem) if rem else None
+        g_warm.replay()
     torch.cuda.synchronize()
     barrier()
     sampler = ClockSampler(clock_gpu) if clock_gpu is not None else None
@@ -280,14 +299,17 @@ def time_graphs(sweep: Sweep, steps: int, warmup: int, stream, clock_gpu: int | 
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             start.record(stream)
-            for s in range(steps):
-                graphs[(warmup + s) % nphase].replay()
+            for _ in range(full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
             end.record(stream)
         torch.cuda.synchronize()
         total_ms = start.elapsed_time(end)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
+    del g_warm, g_full, g_rem
     # per-call breakdown (untimed): external event records between calls
     per_call = [0.0] * sweep.launches_per_step
     with torch.cuda.stream(stream):
@@ -377,14 +399,16 @@ def check_outputs(sweep: Sweep, samples: int = 64):
 def cpu_baseline(seconds: float = 10.0, threads: int | None = None):
     """The oracle (unpack + double-precision layer) on a bounded sample of the
     sweep: for every (shape, M), the first rows of the matrix, sized so the
-    whole sample takes about `seconds`.  Returns packed bytes/s and details."""
+    whole sample takes about `seconds` with all host threads; the same sample
+    is then timed with one thread.  Inputs are packed by the oracle's own
+    codec.  Returns packed bytes/s and details."""
     import oracle
     import synth
     o = oracle.get()
     threads = threads or os.cpu_count() or 1
     # calibrate on a small slice
     K, N = SWEEP[0]
-    P, T, alpha = make_matrix(2, K, 64, 0)
+    P, T, alpha = make_matrix(2, K, 64, 0, codec="oracle")
     X = synth.activations(0, 8, K)
     t0 = time.perf_counter()
     rc, Tu, _ = o.unpack(2, P, K)
@@ -392,23 +416,35 @@ def cpu_baseline(seconds: float = 10.0, threads: int | None = None):
     per_trit_m = (time.perf_counter() - t0) / (64 * K * 8)
     total_trit_m = sum(K * N for (K, N) in SWEEP) * sum(SWEEP_M)
     frac = min(1.0, seconds / max(per_trit_m * total_trit_m, 1e-9))
-    done_bytes, elapsed, rows_used = 0, 0.0, []
+    mats, rows_used = [], []
     for i, (K, N) in enumerate(SWEEP):
-        rows = max(threads, int(N * frac))
-        rows = min(rows, N)
-        Pm, Tm, alpha = make_matrix(2, K, rows, i)
-        for M in SWEEP_M:
-            X = synth.activations(i, M, K)
-            t0 = time.perf_counter()
-            rc, Tu, _ = o.unpack(2, Pm, K)
-            o.linear(Tu, X, alpha, nthreads=threads)
-            elapsed += time.perf_counter() - t0
-            done_bytes += rows * ((K + 3) // 4)
+        rows = min(N, max(threads, int(N * frac)))
+        Pm, _, alpha = make_matrix(2, K, rows, i, codec="oracle")
+        mats.append((K, rows, Pm, alpha, {M: synth.activations(i, M, K) for M in SWEEP_M}))
         rows_used.append(rows)
-    return {"value": round(done_bytes / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads,
+
+    def timed(nthreads, sample):
+        done, el = 0, 0.0
+        for (K, rows, Pm, alpha, xs) in sample:
+            for M in SWEEP_M:
+                t0 = time.perf_counter()
+                rc, Tu, _ = o.unpack(2, Pm, K)
+                o.linear(Tu, xs[M], alpha, nthreads=nthreads)
+                el += time.perf_counter() - t0
+                done += rows * ((K + 3) // 4)
+        return done, el
+
+    done, elapsed = timed(threads, mats)
+    # one thread: a twentieth of the rows (the rate is per byte)
+    small = [(K, max(1, rows // 20), Pm[:max(1, rows // 20)], a, xs)
+             for (K, rows, Pm, a, xs) in mats]
+    done1, el1 = timed(1, small)
+    return {"value": round(done / elapsed / 1e9, 4), "unit": "GB/s", "cores": threads,
             "kind": "oracle",
             "sample": f"first {rows_used} rows of each sweep matrix (both M), unpack + double "
-                      f"accumulation, {elapsed:.1f} s"}
+                      f"accumulation, {elapsed:.1f} s",
+            "one_thread": {"value": round(done1 / el1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                           "sample": f"first {[m[1] for m in small]} rows, {el1:.1f} s"}}
 
 
 def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: int = 3):
@@ -430,19 +466,23 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     out = {}
 
     def timed(plan):
+        # one graph holds `steps` consecutive decode steps (each one launch over
+        # the 210 layers, chained by programmatic dependent launch)
         with torch.cuda.stream(stream):
             tl.gemv_batch_run(plan, stream=stream, flags=1)
             torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
+            gw, g = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gw, stream=stream):
+                for _ in range(warmup):
+                    tl.gemv_batch_run(plan, stream=stream, flags=1)
             with torch.cuda.graph(g, stream=stream):
-                tl.gemv_batch_run(plan, stream=stream, flags=1)
-            for _ in range(warmup):
-                g.replay()
+                for _ in range(steps):
+                    tl.gemv_batch_run(plan, stream=stream, flags=1)
+            gw.replay()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
             a.record(stream)
-            for _ in range(steps):
-                g.replay()
+            g.replay()
             b.record(stream)
             torch.cuda.synchronize()
         return a.elapsed_time(b) / steps
@@ -552,15 +592,30 @@ def secondary(dev, stream, quick: bool):
     import ternary_weight_03_b200 as tl
     out = {}
     pk = peaks()
-    # 1.6-bit sweep, one launch per step
-    sw = Sweep(16, dev)
-    sw.use_batch()
-    ms, per_launch, _ = time_graphs(sw, 5, 3, stream)
-    gbs = sw.bytes_per_step * 5 / (ms * 1e-3) / 1e9
-    out["gemv_1p6bit_sweep"] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
-                                "ms_per_step": round(ms / 5, 4)}
-    del sw
-    torch.cuda.empty_cache()
+    # the 2-bit sweep at one token count only (M = 1: the decode GEMV of a
+    # single sequence), one launch per step
+    for ms_, key in (((1,), "gemv_2bit_sweep_M1"), ((8,), "gemv_2bit_sweep_M8")):
+        sw = Sweep(2, dev, ms=ms_)
+        sw.use_batch()
+        n = 90
+        ms, _, _ = time_graphs(sw, n, 5, stream)
+        gbs = sw.bytes_per_step * n / (ms * 1e-3) / 1e9
+        out[key] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+                    "us_per_step": round(ms / n * 1e3, 2), "packed_bytes": sw.bytes_per_step}
+        del sw
+        torch.cuda.empty_cache()
+    # 1.6-bit sweep (config 3) at three trit sparsities, one launch per step
+    for p0 in (0.2, 1.0 / 3.0, 0.6):
+        sw = Sweep(16, dev, p0=p0)
+        sw.use_batch()
+        n = 45
+        ms, per_launch, _ = time_graphs(sw, n, 5, stream)
+        gbs = sw.bytes_per_step * n / (ms * 1e-3) / 1e9
+        out[f"gemv_1p6bit_sweep_p0_{p0:.2f}"] = {
+            "GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
+            "us_per_step": round(ms / n * 1e3, 2)}
+        del sw
+        torch.cuda.empty_cache()
     # batched GEMM, both formats
     import synth
     for fmt, key in ((2, "gemm_2bit"), (16, "gemm_1p6bit")):
@@ -568,7 +623,7 @@ def secondary(dev, stream, quick: bool):
         for (K, N) in ((4096, 14336), (14336, 4096)):
             P, _, alpha = make_matrix(fmt, K, N, 0)
             dP = torch.from_numpy(P).to(dev)
-            for M in ((16, 256, 4096) if quick else (16, 64, 256, 1024, 4096)):
+            for M in (16, 64, 256, 1024, 4096):
                 X = torch.from_numpy(synth.activations(1, M, K)).to(dev)
                 Y = torch.empty((M, N), dtype=torch.float16, device=dev)
 
@@ -610,10 +665,10 @@ def secondary(dev, stream, quick: bool):
     # the same 2-bit sweep as twelve tl_gemv_ex calls per step (with and without PDL)
     sw = Sweep(2, dev)
     for flags, key in ((1, "gemv_2bit_sweep_per_call_pdl"), (0, "gemv_2bit_sweep_per_call")):
-        ms, _, _ = time_graphs(sw, 20, 3, stream, flags=flags)
-        gbs = sw.bytes_per_step * 20 / (ms * 1e-3) / 1e9
+        ms, _, _ = time_graphs(sw, 45, 3, stream, flags=flags)
+        gbs = sw.bytes_per_step * 45 / (ms * 1e-3) / 1e9
         out[key] = {"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 4),
-                    "us_per_step": round(ms / 20 * 1e3, 2)}
+                    "us_per_step": round(ms / 45 * 1e3, 2)}
     return out
 
 
@@ -669,14 +724,15 @@ def run_gpu(args):
             "launches_per_step": sweep.launches_per_step,
             "l2": f"inputs larger than L2: {sweep.copies} rotating copies of the packed "
                   f"matrices ({sweep.rotation_bytes / 2**20:.0f} MiB) so every call reads HBM",
-            "timing": "CUDA graph per step, CUDA events on the launch stream",
+            "timing": f"CUDA graphs of up to {GRAPH_STEPS} consecutive steps, CUDA events on "
+                      "the launch stream",
             "launch": "one tl_gemv_batch_run per step (all 12 independent layers in one "
                       "persistent launch) with TL_FLAG_PDL",
             "parallelism": f"replicas x{world}",
         },
         "roofline": {
             "bound": "hbm",
-            "kernel": "tlk::gemvp_kernel<2>",
+            "kernel": "tlk::decode2_kernel",
             "achieved": round(achieved, 2),
             "peak": pk["hbm_gbs"],
             "unit": "GB/s",
@@ -711,7 +767,7 @@ def run_gpu(args):
 def traffic_per_launch():
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel sources (else None)."""
-    p = ROOT / "profiles" / "gemvp2_sweep_traffic.json"
+    p = ROOT / "profiles" / "decode2_sweep_traffic.json"
     if not p.exists():
         return None
     try:
@@ -743,7 +799,7 @@ def run_reference(args):
     # that warmup + steps take about a minute in total
     budget_s = 60.0 / max(1, args.steps + args.warmup)
     K, N = SWEEP[0]
-    P, T, alpha = make_matrix(2, K, 64, 0)
+    P, T, alpha = make_matrix(2, K, 64, 0, codec="oracle")
     X = synth.activations(0, 8, K)
     t0 = time.perf_counter()
     o.linear(o.unpack(2, P, K)[1], X, alpha, nthreads=threads)
@@ -752,7 +808,7 @@ def run_reference(args):
     mats = []
     for i, (K, N) in enumerate(SWEEP):
         rows = min(N, max(threads, int(N * frac)))
-        Pm, _, alpha = make_matrix(2, K, rows, i)
+        Pm, _, alpha = make_matrix(2, K, rows, i, codec="oracle")
         mats.append((K, rows, Pm, alpha, {M: synth.activations(i, M, K) for M in SWEEP_M}))
     step_bytes = sum(rows * ((K + 3) // 4) for (K, rows, _, _, _) in mats) * len(SWEEP_M)
 

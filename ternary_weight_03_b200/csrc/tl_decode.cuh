@@ -38,7 +38,8 @@
 // units (unit u by converting warp u mod their number) into the workspace
 // and counts them per layer; a stage's converted operands then arrive by one
 // bulk copy next to its weights.  Layers flagged as reading an earlier
-// layer's output (their X is written during this launch) are converted per
+// layer's output (their X is written during this launch), and the first item
+// of every CTA (so no CTA starts by waiting for others), are converted per
 // item instead, from X in global memory, by stager warps.
 //
 // Warp roles of a CTA (768 threads):
@@ -264,17 +265,20 @@ __device__ __forceinline__ bool dk_wait_count(const uint32_t *p, uint32_t target
     if ((threadIdx.x & 31) == 0) {
         const uint64_t t0 = globaltimer_ns();
         while (true) {
-            if (all_p && dk_ld_acquire(all_p) >= all_target) {
+            // both counters are read before either is tested (one round trip per poll)
+            const uint32_t va = all_p ? dk_ld_acquire(all_p) : 0u;
+            const uint32_t vp = dk_ld_acquire(p);
+            if (all_p && va >= all_target) {
                 all = true;
                 break;
             }
-            if (dk_ld_acquire(p) >= target) break;
+            if (vp >= target) break;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 atomicOr(&g_error_word, kErrTimeout);
                 good = false;
                 break;
             }
-            __nanosleep(64);
+            __nanosleep(32);
         }
     }
     all = __shfl_sync(0xffffffffu, all ? 1 : 0, 0) != 0;
@@ -522,7 +526,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 break;
             }
             const bool valid = item < a.total_items;
-            const bool pre = valid && R.B != nullptr;
+            // the CTA's first item is converted on chip by the stagers (integer
+            // engine: one or two tokens per stage), so the CTA starts without
+            // waiting for other CTAs' conversions
+            const bool pre = valid && R.B != nullptr && (waited || R.M > kDkImmaMaxM);
             if (lane == 0) {
                 DkQEntry e{};
                 e.item = valid ? item : -1;
@@ -666,7 +673,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
     } else if (warp < kDkFirstEpi) {
         // ---------------- stagers ----------------
         // Stages whose operands were converted beforehand pass them by; the
-        // others (chained layers) are converted here from X
+        // others (a CTA's first item, chained layers) are converted here from X
         // in global memory once the stage's weights have landed -- after the
         // producer's wait for the inputs, so X is final.  A stage's weights
         // arriving also means the consumers have released the slot's previous
@@ -1116,17 +1123,21 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
 // ---- host side ---------------------------------------------------------------
 namespace tlk {
 
-// Stages per item for a batch of `total` stages: about six items per SM of a
-// B200, so the last items leave little tail, but between 8 and 16 stages
-// (4096 to 8192 trits of K), so item boundaries (and the epilogue work per
-// item) stay rare.
-inline int dk_item_stages(int64_t total) {
-    const int64_t t = total / (6 * kDkRefSms);
-    return t < 8 ? 8 : (t > 16 ? 16 : (int)t);
+// Relative cost of a stage: the fp16 engine (M >= 3) takes about twice as
+// long per stage as the integer engine.
+inline int dk_stage_cost(int M) { return M <= kDkImmaMaxM ? 1 : 2; }
+// Cost per item for a batch of total cost `total` (in integer-engine stages):
+// about four items per SM of a B200, so that the longest-first order leaves a
+// short tail, but 4..16 integer-engine stages of cost, so item boundaries
+// (and the epilogue work per item) stay rare.
+inline int dk_item_cost(int64_t total) {
+    const int64_t t = total / (4 * kDkRefSms);
+    return t < 4 ? 4 : (t > 16 ? 16 : (int)t);
 }
 // K-parts of a layer: items of about `target` stages, cut at stage
 // boundaries, never more than kDkMaxItemStages stages per item.
 inline int dk_parts(int stages, int target) {
+    if (target < 1) target = 1;
     int parts = (stages + target / 2) / target;
     if (parts < 1) parts = 1;
     while ((stages + parts - 1) / parts > kDkMaxItemStages) ++parts;
@@ -1163,12 +1174,19 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     };
     int64_t total = 0;
     for (int l = 0; l < count; ++l)
-        total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows);
-    const int target = dk_item_stages(total);
+        total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows) *
+                 dk_stage_cost(in[l].M);
+    const int cost = dk_item_cost(total);
+    // fp16-engine items stay at 8 stages or more: their epilogue (M outputs
+    // per row) must keep up with the consumers
+    auto target_of = [&](const DkHostLayer &h) {
+        const int t = cost / dk_stage_cost(h.M);
+        return h.M > kDkImmaMaxM && t < 8 ? 8 : t;
+    };
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
         const int stages = stages_of(h);
-        const int parts = dk_parts(stages, target);
+        const int parts = dk_parts(stages, target_of(h));
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         sc.total_items += tiles * parts;
         sc.total_tiles += tiles;
@@ -1189,7 +1207,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
         const int stages = stages_of(h);
-        const int parts = dk_parts(stages, target);
+        const int parts = dk_parts(stages, target_of(h));
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         const int bstride = kDkMetaBytes + (int)dk_stage_b(h.M);
         uint8_t *B = h.reads_earlier ? nullptr : ws + wl.staged + staged;
@@ -1237,11 +1255,11 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         tile_begin += tiles;
     }
     // Items are handed out in table order.  Without dependencies between
-    // layers, the longest items go first, so the last ones handed out (the
-    // launch's tail) are the shortest.
+    // layers, the costliest items go first, so the last ones handed out (the
+    // launch's tail) are the cheapest.
     if (!sc.chained)
         std::stable_sort(items->begin(), items->end(), [](const DkItemRec &x, const DkItemRec &y) {
-            return x.s1 - x.s0 > y.s1 - y.s0;
+            return (x.s1 - x.s0) * dk_stage_cost(x.M) > (y.s1 - y.s0) * dk_stage_cost(y.M);
         });
     return sc;
 }

@@ -111,16 +111,20 @@ def _up(v):
 def _ws2_expected(layers):
     """2-bit batch workspace, region by region (each rounded up to 256 bytes):
     counters, one 128-byte tensor map per layer, a 96-byte record per work item
-    (256-row tile x K-part of 8..16 stages of 512 trits), a 48-byte record per
+    (256-row tile x K-part of 2..16 stages of 512 trits), a 48-byte record per
     conversion unit (stage x token of a layer that reads no earlier output), a
     u32 per layer and per tile, 8-byte partials of split tiles, and the
     converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage)."""
     items = units = tiles = slots = staged = 0
     stg = lambda d: -(-(-(-d["K"] // 4)) // 128)
-    total = sum(stg(d) * -(-d["N"] // 256) for d in layers)
-    target = min(16, max(8, total // (6 * 148)))  # stages per item
+    cm = lambda d: 1 if d["M"] <= 2 else 2  # relative cost of a stage
+    total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
+    cost = min(16, max(4, total // (4 * 148)))  # cost per item
     for d in layers:
         stages = stg(d)
+        target = max(1, cost // cm(d))
+        if d["M"] > 2:
+            target = max(target, 8)
         parts = max(1, min(stages, (stages + target // 2) // target))
         t = -(-d["N"] // 256)
         items += t * parts
