@@ -94,7 +94,7 @@ constexpr int kDkMetaBytes = 64;                        // per stage: per-token 
 // Workspace counters (u32 words of the 256-byte header).
 constexpr int kDkCtrFinal = 1;      // tiles whose outputs are stored
 constexpr int kDkCtrDone = 2;       // CTAs that have finished
-constexpr int kDkCtrItems = 3;      // items handed out beyond the first gridDim.x
+constexpr int kDkCtrItems = 3;      // items handed out beyond the first 2 gridDim.x
 constexpr int kDkCtrUnitsDone = 5;  // CTAs whose conversion units are all written
 
 // Bytes of converted B operands of one stage of a layer with M tokens: the
@@ -184,7 +184,9 @@ struct DkQEntry {
     float alpha;
     int item;  // -1: no more items
     int tile, part, s0, s1, M, K, N, ldx, ldy, parts, tile_begin;
-    int pre;   // 1: converted operands arrive with the weights; 0: a stager converts X
+    int pre;      // 1: converted operands arrive with the weights; 0: a stager converts X
+    int chained;  // X is written by earlier layers of this launch
+    int pad_;
 };
 
 struct DkLayout {
@@ -550,6 +552,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     e.parts = R.parts;
                     e.tile_begin = R.tile_begin;
                     e.pre = pre ? 1 : 0;
+                    e.chained = R.wait_tiles > 0 ? 1 : 0;
                 }
                 queue[q] = e;
                 mbar_arrive(&qfull[q]);
@@ -606,10 +609,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 }
                 pdl_wait();
                 waited = true;
-                // the counter was reset by the previous grid's last CTA
-                int nx = 0;
-                if (lane == 0) nx = G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
-                next = __shfl_sync(0xffffffffu, nx, 0);
+                // the second item is static too (blockIdx.x + G): no counter round
+                // trip before the CTA's first stages; later ones come from the
+                // counter, which the previous grid's last CTA reset
+                next = item + G;
                 const bool in_ok = wait_inputs();
                 if (lane == 0) {
                     for (int i = 0; i < pre_n; ++i) {
@@ -641,7 +644,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             if (next < a.total_items) NR = dk_load_rec<DkItemRec, 6>(a.items, next);
             int nx2 = 0;
             if (lane == 0 && next < a.total_items)
-                nx2 = G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
+                nx2 = 2 * G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
             for (; s < R.s1; ++s, ++stage) {
                 const int slot = ps;
                 if (wrapped && !dk_warp_wait(&empty[slot], pph ^ 1u)) {
@@ -674,13 +677,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         // ---------------- stagers ----------------
         // Stages whose operands were converted beforehand pass them by; the
         // others (a CTA's first item, chained layers) are converted here from X
-        // in global memory once the stage's weights have landed -- after the
-        // producer's wait for the inputs, so X is final.  A stage's weights
-        // arriving also means the consumers have released the slot's previous
-        // round, so xfull is never arrived on a round ahead.
+        // in global memory.  xfull is never arrived on a round ahead: a slot's
+        // round r >= 1 starts only once the consumers released round r - 1.
         const int sw = warp - 1;
         int ss = 0;
         uint32_t sph = 0;
+        bool first_round = true;  // no earlier use of any slot to wait out
         int qi = 0;
         bool ok = true;
         DkQEntry e;
@@ -689,12 +691,26 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             for (int s = e.s0; s < e.s1; ++s) {
                 const int slot = ss;
                 const uint32_t ph = sph;
+                const bool fresh = first_round;
                 if (++ss == NS) {
                     ss = 0;
                     sph ^= 1u;
+                    first_round = false;
                 }
                 if (e.pre || slot % kDkStagers != sw) continue;  // converted, or another stager's
-                if (!dk_warp_wait(&wfull[slot], ph)) {
+                // A slot's first use needs no wait (X of a layer without
+                // dependencies is final since pdl_wait).  A later use waits for the
+                // consumers to release the slot's previous round: on `empty`, not on
+                // the weights of this round -- a stager that skipped its first-round
+                // wait may reach round 1 while the slot is still in phase 0, and a
+                // parity wait on wfull would then pass a phase early.  Chained
+                // layers also wait for this round's weights, which the producer
+                // issues only once it has seen X final.
+                if (!fresh && !dk_warp_wait(&empty[slot], ph ^ 1u)) {
+                    ok = false;
+                    break;
+                }
+                if (e.chained && !dk_warp_wait(&wfull[slot], ph)) {
                     ok = false;
                     break;
                 }
@@ -729,31 +745,78 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             int64_t *slot = e.parts > 1 ? a.partials + e.part_off +
                                               (int64_t)(e.tile * e.parts + e.part) * cnt
                                         : nullptr;
-            // partial of (token m, warp cw, tile pair tile t, MMA row rho) at
+            // partial of (token m, warp cw, tile t of the warp, MMA row rho) at
             // ((m*16 + cw)*2 + t)*16 + rho; the two warps of a row tile (cw, cw + 8)
-            // are 256 entries apart, and 32 consecutive rows of one token read 32
-            // consecutive entries
-            for (int idx = lane; idx < cnt; idx += 32) {
-                const int r = idx % kDkRows, m = idx / kDkRows;  // consecutive lanes: consecutive n
-                const int t = r >> 4, tp = t >> 1, tl = t & 1;
-                const int rho = (r & 8) + dk_pi_inv(r & 7);
-                const int base = ((m * 16 + tp) * 2 + tl) * 16 + rho;
+            // are 256 entries apart.  A lane takes 8 consecutive rows r0 .. r0 + 7
+            // of one token: MMA rows (r0 & 8) + pi^-1(0..7), 8 consecutive entries.
+            for (int gi = lane; gi < cnt / 8; gi += 32) {
+                const int m = gi / (kDkRows / 8), r0 = (gi % (kDkRows / 8)) * 8;
+                const int t = r0 >> 4, tp = t >> 1, tl = t & 1;
+                const int base = ((m * 16 + tp) * 2 + tl) * 16 + (r0 & 8);
+                float y[8];
+                int64_t iv[8];
                 if (exact) {
-                    const int64_t *p = reinterpret_cast<const int64_t *>(pb);
-                    const int64_t v = p[base] + p[base + 256];
-                    if (slot) {
-                        slot[idx] = v;
-                    } else if (n0 + r < e.N) {
-                        const double y = (double)e.alpha * ((double)v * 5.9604644775390625e-8);
-                        e.Y[(int64_t)m * e.ldy + n0 + r] = __half_as_ushort(__double2half(y));
+                    const int64_t *p = reinterpret_cast<const int64_t *>(pb) + base;
+#pragma unroll
+                    for (int q = 0; q < 8; q += 2) {
+                        const longlong2 u = *reinterpret_cast<const longlong2 *>(p + q);
+                        const longlong2 w = *reinterpret_cast<const longlong2 *>(p + 256 + q);
+                        iv[dk_pi(q)] = u.x + w.x;  // MMA row q holds physical row pi(q)
+                        iv[dk_pi(q + 1)] = u.y + w.y;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        y[j] = (float)((double)e.alpha * ((double)iv[j] * 5.9604644775390625e-8));
+                } else {
+                    const float *p = reinterpret_cast<const float *>(pb) + base;
+                    const float4 u0 = *reinterpret_cast<const float4 *>(p);
+                    const float4 u1 = *reinterpret_cast<const float4 *>(p + 4);
+                    const float4 w0 = *reinterpret_cast<const float4 *>(p + 256);
+                    const float4 w1 = *reinterpret_cast<const float4 *>(p + 260);
+                    const float v[8] = {u0.x + w0.x, u0.y + w0.y, u0.z + w0.z, u0.w + w0.w,
+                                        u1.x + w1.x, u1.y + w1.y, u1.z + w1.z, u1.w + w1.w};
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) y[dk_pi(q)] = v[q];
+                }
+                const int idx0 = m * kDkRows + r0;
+                if (slot) {
+                    // this part's partial of a split tile (int64 or double bits)
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        longlong2 o;
+                        if (exact) {
+                            o.x = iv[j];
+                            o.y = iv[j + 1];
+                        } else {
+                            o.x = __double_as_longlong((double)y[j]);
+                            o.y = __double_as_longlong((double)y[j + 1]);
+                        }
+                        *reinterpret_cast<longlong2 *>(slot + idx0 + j) = o;
                     }
                 } else {
-                    const float *p = reinterpret_cast<const float *>(pb);
-                    const float v = p[base] + p[base + 256];
-                    if (slot) {
-                        reinterpret_cast<double *>(slot)[idx] = (double)v;
-                    } else if (n0 + r < e.N) {
-                        e.Y[(int64_t)m * e.ldy + n0 + r] = f32_to_f16_bits(e.alpha * v);
+                    // fp16_rn(alpha * v): exact items round once from double
+                    uint32_t h[4];
+#pragma unroll
+                    for (int j = 0; j < 8; j += 2) {
+                        uint16_t lo, hi;
+                        if (exact) {
+                            lo = __half_as_ushort(__double2half(
+                                (double)e.alpha * ((double)iv[j] * 5.9604644775390625e-8)));
+                            hi = __half_as_ushort(__double2half(
+                                (double)e.alpha * ((double)iv[j + 1] * 5.9604644775390625e-8)));
+                        } else {
+                            lo = f32_to_f16_bits(e.alpha * y[j]);
+                            hi = f32_to_f16_bits(e.alpha * y[j + 1]);
+                        }
+                        h[j / 2] = (uint32_t)lo | ((uint32_t)hi << 16);
+                    }
+                    uint16_t *yr = e.Y + (int64_t)m * e.ldy + n0 + r0;
+                    if (n0 + r0 + 8 <= e.N) {
+                        *reinterpret_cast<uint4 *>(yr) = make_uint4(h[0], h[1], h[2], h[3]);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            if (n0 + r0 + j < e.N) yr[j] = (uint16_t)(h[j / 2] >> (16 * (j & 1)));
                     }
                 }
             }
