@@ -236,6 +236,18 @@ int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
  * TL_ERR_CUDA. */
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream);
 
+/* Failure-detection hook of tl_gemv_batch_run, honoured only by the debug
+ * library (libternary_debug.so, the same sources compiled with
+ * TL_DEBUG_HOOKS); the product library rejects the bit with
+ * TL_ERR_INVALID_ARG.  With it, the 2-bit batch kernel's CTA 0 leaves out
+ * the shared-memory barrier arrival that publishes its first operand stage
+ * converted on chip (a batch whose first item has M <= 2).  Its consumers'
+ * bounded wait then runs out: every warp of the launch gives up its work
+ * within the wait limit (1 s), the CTA waits for its own copies in flight
+ * and exits, and tl_device_status returns TL_ERR_TIMEOUT.  No hardware
+ * completion is ever skipped. */
+#define TL_FLAG_DEBUG_DROP_ARRIVE 0x80000000u
+
 /* Batched / prefill-shaped layer, M >= TL_GEMM_MIN_M, same arguments and
  * rules as tl_gemv, both formats ("Pith review of Spectra 1.1", "What carries
  * the argument": an FP16 x INT2 tensor-core kernel with fused dequantisation;

@@ -17,6 +17,7 @@ import numpy as np
 
 PKG = Path(__file__).resolve().parent
 LIB_PATH = PKG / "libternary.so"
+DEBUG_LIB_PATH = PKG / "libternary_debug.so"
 
 FMT_2BIT = 2
 FMT_1P6BIT = 16
@@ -81,22 +82,37 @@ class TLError(RuntimeError):
 
 
 _lib = None
+_debug_lib = None
+
+
+def _load(path: Path) -> ctypes.CDLL:
+    if not path.exists():
+        raise RuntimeError(f"{path.name} not found at {path}: run "
+                           "`python -m ternary_weight_03_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(str(path))
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
 
 
 def lib() -> ctypes.CDLL:
     """The loaded libternary.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not LIB_PATH.exists():
-            raise RuntimeError(f"libternary.so not found at {LIB_PATH}: run "
-                               "`python -m ternary_weight_03_b200.build` (nvcc, sm_100a)")
-        L = ctypes.CDLL(str(LIB_PATH))
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(L, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = L
+        _lib = _load(LIB_PATH)
     return _lib
+
+
+def debug_lib() -> ctypes.CDLL:
+    """libternary_debug.so: the same entry points, plus the failure-detection
+    hook TL_FLAG_DEBUG_DROP_ARRIVE of tl_gemv_batch_run.  Its device error word
+    is its own (read it with its tl_device_status)."""
+    global _debug_lib
+    if _debug_lib is None:
+        _debug_lib = _load(DEBUG_LIB_PATH)
+    return _debug_lib
 
 
 def _check(fn: str, rc: int):
@@ -157,6 +173,7 @@ def _stream_ptr(stream) -> int:
 
 
 FLAG_PDL = 1
+FLAG_DEBUG_DROP_ARRIVE = 0x80000000  # debug library only
 
 
 def _layer(fn_name: str, fmt: int, dT, alpha: float, X, K: int, out=None, stream=None, M=None,

@@ -175,6 +175,7 @@ struct DkArgs {
     int total_units;
     int maxM;
     int chained;  // some layer reads an earlier layer's output
+    int drop_arrive;  // failure-detection hook (debug library only), else 0
 };
 
 struct DkQEntry {
@@ -723,6 +724,11 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     else
                         dk_conv_hmma(src, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
                 }
+#ifdef TL_DEBUG_HOOKS
+                // the hook: CTA 0's first stage converted here is never published
+                if (a.drop_arrive && blockIdx.x == 0 && s == e.s0 && e.item == (int)blockIdx.x)
+                    continue;
+#endif
                 mbar_arrive(&xfull[slot]);
             }
         }
@@ -1360,6 +1366,7 @@ inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int
     a.total_units = total_units;
     a.maxM = maxM;
     a.chained = chained;
+    a.drop_arrive = 0;
     return a;
 }
 
@@ -1398,7 +1405,7 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     cfg.attrs = at;
     cfg.numAttrs = pdl ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, decode2_kernel, a);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;
         return 5;

@@ -211,7 +211,7 @@ int tl_gemv_ex(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint1
         e = cudaLaunchKernelEx(&cfg, tlk::gemv_kernel<16>, dT, ldp, alpha, dX, ldx, dY, ldy, M,
                                (int)N, (int)K, sh.tiles_per_cta);
     }
-    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) return cuda_fail(e);
     return TL_OK;
 }
@@ -328,7 +328,12 @@ int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
 
 int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream) {
     if (!plan || !plan->dWorkspace) return TL_ERR_INVALID_ARG;
-    if (flags & ~(unsigned int)TL_FLAG_PDL) return TL_ERR_INVALID_ARG;
+#ifdef TL_DEBUG_HOOKS
+    constexpr unsigned int kRunFlags = TL_FLAG_PDL | TL_FLAG_DEBUG_DROP_ARRIVE;
+#else
+    constexpr unsigned int kRunFlags = TL_FLAG_PDL;
+#endif
+    if (flags & ~kRunFlags) return TL_ERR_INVALID_ARG;
     if (plan->fmt != TL_FMT_2BIT && plan->fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
     if (plan->count < 1 || plan->count > TL_GEMV_BATCH_MAX || plan->max_m < 1 ||
         plan->max_m > TL_GEMV_MAX_M || plan->total_items < 1 || plan->total_tiles < 1 ||
@@ -349,9 +354,10 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
     }
     const bool pdl = (flags & TL_FLAG_PDL) != 0;
     if (plan->fmt == TL_FMT_2BIT) {
-        const tlk::DkArgs da =
+        tlk::DkArgs da =
             tlk::dk_args(plan->dWorkspace, plan->count, plan->total_items, plan->total_units,
                          plan->total_tiles, plan->max_m, plan->chained);
+        da.drop_arrive = (flags & TL_FLAG_DEBUG_DROP_ARRIVE) ? 1 : 0;
         return tlk::launch_decode2(da, dev->num_sms, pdl, (cudaStream_t)stream, &t_last_cuda_error);
     }
     const tlk::GpArgs a = tlk::gp_args(plan->dWorkspace, plan->count, plan->total_items,

@@ -552,7 +552,7 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
     cfg.attrs = at;
     cfg.numAttrs = S > 1 ? 1 : 0;  // S = 1: a plain launch
     cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_kernel<FMT, BN>, tw, tx, alpha, dY, ldy, M, N, K);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;
         return 5;

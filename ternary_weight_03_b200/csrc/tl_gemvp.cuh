@@ -797,7 +797,7 @@ inline int launch_gemvp(const GpArgs &a, int num_sms, bool pdl, cudaStream_t str
     cfg.attrs = at;
     cfg.numAttrs = pdl ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, gemvp_kernel<FMT>, a);
-    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;
         return 5;

@@ -212,6 +212,7 @@ inline int launch_ternarise(int fmt, const uint16_t *dW, int64_t ldw, int N, int
     int g1 = 4 * num_sms;
     if (g1 > kTzMaxPartials) g1 = kTzMaxPartials;
     if (steps1 < g1) g1 = (int)steps1;
+    (void)cudaGetLastError();  // an error of an earlier call was returned by that call
     absum_kernel<<<g1, kTzThreads, 0, stream>>>(dW, ldw, N, K, partials);
     scale_kernel<<<1, kTzThreads, 0, stream>>>(partials, g1, (int64_t)N * K, dAlpha);
     const int words = (int)(ldp / 4);

@@ -31,6 +31,27 @@ def test_every_declared_symbol_is_exported(L):
     assert set(names) == set(tl.SIGNATURES), "binding and header disagree"
 
 
+def test_only_the_c_abi_is_exported(L):
+    """Both libraries export nothing but tl_* symbols: no C++ function-local
+    static (process-unique symbol) is shared between two of them loaded into
+    one process."""
+    import shutil
+    import subprocess
+    if shutil.which("readelf") is None:
+        pytest.skip("readelf not available")
+    for lib in (tlbuild.LIB, tlbuild.DEBUG_LIB):
+        out = subprocess.run(["readelf", "--dyn-syms", "-W", str(lib)], check=True,
+                             capture_output=True, text=True).stdout
+        defined = []
+        for line in out.splitlines():
+            f = line.split()
+            if len(f) >= 8 and f[0][:-1].isdigit() and f[6] != "UND":
+                defined.append((f[4], f[7]))
+        assert defined, lib
+        bad = [d for d in defined if not d[1].startswith("tl_") or d[0] == "UNIQUE"]
+        assert not bad, f"{lib.name} exports {bad[:5]}"
+
+
 def test_status_strings(L):
     for code, name in tl.STATUS.items():
         assert tl.status_str(code).startswith(name)

@@ -36,6 +36,20 @@ def test_small_ragged(fmt, M, N, K):
     check_against_oracle(T, X, a, Y)
 
 
+# Rows longer than one cluster of the single-layer kernel stages (2-bit
+# K > 16384, 1.6-bit K > 20480) go to the register-streaming kernel: ragged N,
+# K with a tail inside a byte, both token extremes, junk padding, repeat calls.
+LONG_K = [(2, 1, 300, 20000), (2, 8, 77, 20000), (2, 3, 129, 40001),
+          (16, 1, 300, 24000), (16, 8, 77, 24000), (16, 5, 33, 65537)]
+
+
+@pytest.mark.parametrize("fmt,M,N,K", LONG_K)
+def test_long_rows(fmt, M, N, K):
+    T, X, a = make_case(fmt, M, N, K, seed=K + N, p0=[0.2, 1 / 3, 0.6][N % 3])
+    Y, _ = run_layer(fmt, T, X, a, ldx_extra=1, repeat=2)
+    check_against_oracle(T, X, a, Y)
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("extra", [(1, 0, 0), (0, 2, 0), (0, 0, 3), (2, 1, 1)])
 def test_strides(fmt, extra):
