@@ -884,6 +884,22 @@ def run_batch_once(fmt: int, M: int, reps: int = 3):
                       "checksum": float(sum(sp[4].float().abs().sum() for sp in specs))}))
 
 
+def run_ternarise_once(fmt: int, N: int, K: int, reps: int = 3):
+    """tl_ternarise on one seeded N x K fp16 weight matrix, `reps` times,
+    nothing else on the device (for ncu)."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    from ternary_weight_03_b200 import build
+    build.build()
+    g = torch.Generator(device="cuda").manual_seed(N * 7 + K)
+    W = (torch.randn((N, K), generator=g, device="cuda") * 0.02).half()
+    for _ in range(reps):
+        P, alpha = tl.ternarise(fmt, W)
+    torch.cuda.synchronize()
+    print(json.dumps({"ternarise_once": [fmt, N, K], "alpha": float(alpha.item()),
+                      "checksum": int(P.sum().item())}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -898,7 +914,12 @@ def main(argv=None):
                          "(a small case for profiling the batch kernel)")
     ap.add_argument("--single", metavar="FMT,K,N,M",
                     help="run one seeded layer call 4 times and exit (for ncu captures)")
+    ap.add_argument("--ternarise-once", metavar="FMT,N,K",
+                    help="ternarise one seeded N x K fp16 matrix 3 times and exit (for ncu)")
     args = ap.parse_args(argv)
+    if args.ternarise_once:
+        run_ternarise_once(*[int(v) for v in args.ternarise_once.split(",")])
+        return
     if args.batch_once:
         run_batch_once(*[int(v) for v in args.batch_once.split(",")])
         return

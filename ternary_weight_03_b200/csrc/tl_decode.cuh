@@ -436,6 +436,102 @@ __device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, int valid, int
     if (lane == 0) reinterpret_cast<float *>(meta)[m] = sx;
 }
 
+// The last part of a split tile adds the tile's parts in part order and stores
+// fp16_rn(alpha * sum): int64 partials (integer engine, exact, V * 2^-24) or
+// fp32 partials summed in double.  A lane takes 8 consecutive rows of one
+// token at a time and keeps the loads of several parts in flight.  Not
+// inlined, so its registers do not weigh on the consumer loops.
+__device__ __noinline__ void dk_finalize(const int64_t *base, int cnt, int parts, bool exact,
+                                         float alpha, uint16_t *Y, int64_t ldy, int n0, int N,
+                                         int lane) {
+    for (int gi = lane; gi < cnt / 8; gi += 32) {
+        const int idx0 = gi * 8;  // token idx0 / 256, rows idx0 % 256 ..
+        const int m = idx0 / kDkRows, r0 = idx0 % kDkRows;
+        uint32_t h[4];
+        if (exact) {
+            int64_t acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            int q = 0;
+            for (; q + 2 <= parts; q += 2) {
+                const longlong2 *p0 =
+                    reinterpret_cast<const longlong2 *>(base + (int64_t)q * cnt + idx0);
+                const longlong2 *p1 = reinterpret_cast<const longlong2 *>(
+                    base + (int64_t)(q + 1) * cnt + idx0);
+                longlong2 u[4], w[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    u[j] = __ldcg(p0 + j);
+                    w[j] = __ldcg(p1 + j);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[2 * j] += u[j].x + w[j].x;
+                    acc[2 * j + 1] += u[j].y + w[j].y;
+                }
+            }
+            if (q < parts) {
+                const longlong2 *p0 =
+                    reinterpret_cast<const longlong2 *>(base + (int64_t)q * cnt + idx0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const longlong2 u = __ldcg(p0 + j);
+                    acc[2 * j] += u.x;
+                    acc[2 * j + 1] += u.y;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const uint16_t lo = __half_as_ushort(__double2half(
+                    (double)alpha * ((double)acc[j] * 5.9604644775390625e-8)));
+                const uint16_t hi = __half_as_ushort(__double2half(
+                    (double)alpha * ((double)acc[j + 1] * 5.9604644775390625e-8)));
+                h[j / 2] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+        } else {
+            // fp32 partials, summed in double in part order
+            double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            for (int q0 = 0; q0 < parts; q0 += 4) {
+                const int nq = parts - q0 < 4 ? parts - q0 : 4;
+                float4 u[4][2];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q < nq) {
+                        const float4 *f = reinterpret_cast<const float4 *>(
+                            reinterpret_cast<const float *>(base + (int64_t)(q0 + q) * cnt) +
+                            idx0);
+                        u[q][0] = __ldcg(f);
+                        u[q][1] = __ldcg(f + 1);
+                    }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    if (q < nq) {
+                        acc[0] += u[q][0].x;
+                        acc[1] += u[q][0].y;
+                        acc[2] += u[q][0].z;
+                        acc[3] += u[q][0].w;
+                        acc[4] += u[q][1].x;
+                        acc[5] += u[q][1].y;
+                        acc[6] += u[q][1].z;
+                        acc[7] += u[q][1].w;
+                    }
+            }
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const uint16_t lo = f32_to_f16_bits(alpha * (float)acc[j]);
+                const uint16_t hi = f32_to_f16_bits(alpha * (float)acc[j + 1]);
+                h[j / 2] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+        }
+        uint16_t *yr = Y + (int64_t)m * ldy + n0 + r0;
+        if (n0 + r0 + 8 <= N) {
+            *reinterpret_cast<uint4 *>(yr) = make_uint4(h[0], h[1], h[2], h[3]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (n0 + r0 + j < N) yr[j] = (uint16_t)(h[j / 2] >> (16 * (j & 1)));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
     extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
     const DkLayout lay(a.maxM);
@@ -786,18 +882,17 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 }
                 const int idx0 = m * kDkRows + r0;
                 if (slot) {
-                    // this part's partial of a split tile (int64 or double bits)
+                    // this part's partial of a split tile: int64 entries, or fp32
+                    // entries packed into the first half of the part's region
+                    if (exact) {
 #pragma unroll
-                    for (int j = 0; j < 8; j += 2) {
-                        longlong2 o;
-                        if (exact) {
-                            o.x = iv[j];
-                            o.y = iv[j + 1];
-                        } else {
-                            o.x = __double_as_longlong((double)y[j]);
-                            o.y = __double_as_longlong((double)y[j + 1]);
-                        }
-                        *reinterpret_cast<longlong2 *>(slot + idx0 + j) = o;
+                        for (int j = 0; j < 8; j += 2)
+                            *reinterpret_cast<longlong2 *>(slot + idx0 + j) =
+                                make_longlong2(iv[j], iv[j + 1]);
+                    } else {
+                        float4 *f = reinterpret_cast<float4 *>(reinterpret_cast<float *>(slot) + idx0);
+                        f[0] = make_float4(y[0], y[1], y[2], y[3]);
+                        f[1] = make_float4(y[4], y[5], y[6], y[7]);
                     }
                 } else {
                     // fp16_rn(alpha * v): exact items round once from double
@@ -837,50 +932,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 prev = __shfl_sync(0xffffffffu, prev, 0);
                 final_tile = prev == (uint32_t)(e.parts - 1);
                 if (final_tile) {
-                    // last part of the tile: add the parts in part order
+                    // last part of the tile: add the parts in part order.  A lane
+                    // takes 8 consecutive rows of one token at a time and keeps
+                    // the loads of several parts in flight (16-byte loads).
                     __threadfence();
-                    const int64_t *base = a.partials + e.part_off + (int64_t)e.tile * e.parts * cnt;
-                    for (int i0 = 0; i0 < cnt; i0 += 32 * 4) {
-                        if (exact) {
-                            int64_t acc[4] = {0, 0, 0, 0};
-                            for (int q = 0; q < e.parts; ++q) {
-#pragma unroll
-                                for (int t = 0; t < 4; ++t) {
-                                    const int idx = i0 + lane + 32 * t;
-                                    if (idx < cnt)
-                                        acc[t] += __ldcg(reinterpret_cast<const long long *>(
-                                            base + (int64_t)q * cnt + idx));
-                                }
-                            }
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const int idx = i0 + lane + 32 * t;
-                                const int r = idx % kDkRows, m = idx / kDkRows;
-                                if (idx < cnt && n0 + r < e.N)
-                                    e.Y[(int64_t)m * e.ldy + n0 + r] = __half_as_ushort(__double2half(
-                                        (double)e.alpha * ((double)acc[t] * 5.9604644775390625e-8)));
-                            }
-                        } else {
-                            double acc[4] = {0.0, 0.0, 0.0, 0.0};
-                            for (int q = 0; q < e.parts; ++q) {
-#pragma unroll
-                                for (int t = 0; t < 4; ++t) {
-                                    const int idx = i0 + lane + 32 * t;
-                                    if (idx < cnt)
-                                        acc[t] += __ldcg(reinterpret_cast<const double *>(
-                                            base + (int64_t)q * cnt + idx));
-                                }
-                            }
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const int idx = i0 + lane + 32 * t;
-                                const int r = idx % kDkRows, m = idx / kDkRows;
-                                if (idx < cnt && n0 + r < e.N)
-                                    e.Y[(int64_t)m * e.ldy + n0 + r] =
-                                        f32_to_f16_bits(e.alpha * (float)acc[t]);
-                            }
-                        }
-                    }
+                    dk_finalize(a.partials + e.part_off + (int64_t)e.tile * e.parts * cnt, cnt,
+                                e.parts, exact, e.alpha, e.Y, e.ldy, n0, e.N, lane);
                     if (lane == 0) a.tile_ctr[e.tile_begin + e.tile] = 0u;
                 }
             }
