@@ -12,14 +12,17 @@
 //    (128 rows x 16 B) into a shared-memory ring (no multicast).  A 1.6-bit
 //    row holds 64 trits in 12.8 bytes, so its packed tiles come in blocks of
 //    320 trits (128 rows x 64 B, five K-steps) through a separate 2-deep ring;
-//  * four decode warps (thread = weight row = TMEM lane) expand the row's 64
+//  * sets of four decode warps (four sets for 2-bit, two for 1.6-bit), the
+//    sets taking the K-steps in turn (thread = weight row = TMEM lane),
+//    expand the row's 64
 //    trits to exact fp16 -1 / 0 / +1 and write them with tcgen05.st straight
 //    into tensor memory, where they are the MMA's A operand -- the expanded
 //    weights never touch shared memory;
 //  * one thread issues tcgen05.mma.kind::f16 (A from TMEM, B = activations
 //    from shared memory) into an fp32 accumulator in TMEM and commits to
 //    mbarriers that recycle the ring stages;
-//  * the decode warps then read the accumulator with tcgen05.ld, scale by
+//  * the decode warps then read the accumulator with tcgen05.ld (the sets
+//    taking its 32-column chunks in turn), scale by
 //    alpha and store fp16.
 // Split-K, for shapes with fewer output tiles than SMs: a cluster of S CTAs
 // shares one output tile, rank r taking K-steps [r nk / S, (r + 1) nk / S)
@@ -43,7 +46,17 @@ namespace tlk {
 constexpr int kGemmRows = 128;        // weight rows per tile (TMEM lanes)
 constexpr int kGemmKStep = 64;        // trits per K-step (4 MMAs of K = 16)
 constexpr int kGemmStages = 4;        // ring depth (the A stages in TMEM follow it)
-constexpr int kGemmThreads = 192;     // warp 0 TMA, warp 1 MMA, warps 2..5 decode/epilogue
+// warp 0 TMA, warp 1 MMA, then gemm_dec_sets<FMT> sets of four decode warps
+// (one per TMEM lane quarter); set d takes the K-steps k with k mod sets = d
+// (and the 32-column chunks c of the accumulator with c / 32 mod sets = d in
+// the epilogue).  2-bit: four sets; 1.6-bit: two, since every set reads
+// each packed block whole.
+template <int FMT>
+__host__ __device__ constexpr int gemm_dec_sets() { return FMT == 2 ? 4 : 2; }
+template <int FMT>
+__host__ __device__ constexpr int gemm_threads() { return 64 + 128 * gemm_dec_sets<FMT>(); }
+static_assert(kGemmStages % gemm_dec_sets<2>() == 0 && kGemmStages % gemm_dec_sets<16>() == 0,
+              "each ring stage belongs to one decoder set");
 // TMEM columns: the accumulator takes BN (at least 32) columns, then the four
 // A stages take 32 columns each; the allocation is a power of two.
 __host__ __device__ constexpr int gemm_acol_base(int bn) { return bn < 32 ? 32 : bn; }
@@ -137,10 +150,11 @@ __device__ __forceinline__ void decode16_kstep(int j, const uint32_t (&w)[16], u
 }
 
 template <int FMT, int BN>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads<FMT>(), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
             float alpha, uint16_t *__restrict__ Y, int64_t ldy, int M, int N, int K) {
     using L = GemmSmem<FMT>;
+    constexpr int kGemmDecSets = gemm_dec_sets<FMT>();
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte alignment for the 128-byte-swizzled activation stages
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -182,7 +196,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
         mbar_init(redbar, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&wfull[s], 1);
-            mbar_init(&wempty[s], 128);
+            mbar_init(&wempty[s], 128 * kGemmDecSets);  // every set reads every full block
         }
         // bytes pushed here: (S - 1) sources x the tile's 128 x BN floats / S
         if (S > 1) mbar_arrive_expect_tx(redbar, (S - 1) * (uint32_t)(kGemmRows * BN * 4) / S);
@@ -254,13 +268,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
             tc_commit(done);  // also on abort, so teardown can wait for issued MMAs
         }
     } else {
-        // ---- decode warps (2..5): thread = weight row = TMEM lane ----
+        // ---- decode warps: thread = weight row = TMEM lane; set `half` takes
+        // the K-steps k = half mod kGemmDecSets ----
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;      // row within the tile
+        const int half = (warp - 2) >> 2;
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         bool ok = true;
         uint32_t blk[16];  // 1.6-bit: this row's current 320-trit block
-        for (int k = 0; k < nk && ok; ++k) {
+        int have_blk = -1;  // 1.6-bit: index of the block in blk
+        for (int k = half; k < nk && ok; k += kGemmDecSets) {
             const int s = k % kGemmStages;
             uint32_t a[32];
             if constexpr (FMT == 2) {
@@ -278,8 +295,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             } else {
                 const int j = k % KU;
-                if (j == 0) {
+                if (k / KU != have_blk) {
+                    // this set's first K-step of the block
                     const int b = k / KU, wsl = b & 1;
+                    have_blk = b;
                     ok = mbar_wait(&wfull[wsl], (b >> 1) & 1);
                     if (!ok) break;
                     const uint4 *src = reinterpret_cast<const uint4 *>(
@@ -315,7 +334,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
             tc_fence_after();
             const int n = n0 + row;
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
+            for (int c = 32 * half; c < BN; c += 32 * kGemmDecSets) {
                 uint32_t v[32];
                 tmem_ld_32x32b_x32(tmem + lane_addr + c, v);
                 tc_wait_ld();
@@ -341,13 +360,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
         if (warp >= 2) {
             tc_fence_after();
             const int quarter = warp & 3;
+            const int half = (warp - 2) >> 2;  // the warps of a quarter take chunks in turn
             const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
             const int per = 4 * kChunks / (int)S;  // units owned per rank
             const uint32_t xs_addr = smem_u32(xs);
             // push: unit u = quarter * kChunks + c goes to rank u % S, slot
             // [source rank][u / S][kChunkW / 4 groups of 4 floats][32 lanes]
 #pragma unroll 1
-            for (int c = 0; c < kChunks; ++c) {
+            for (int c = half; c < kChunks; c += kGemmDecSets) {
                 const int u = quarter * kChunks + c;
                 const uint32_t owner = (uint32_t)u % S;
                 if (owner == rank) continue;
@@ -369,7 +389,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
             if (mbar_wait_cluster(redbar, 0)) {
                 const int n = n0 + quarter * 32 + lane;
 #pragma unroll 1
-                for (int c = 0; c < kChunks; ++c) {
+                for (int c = half; c < kChunks; c += kGemmDecSets) {
                     const int u = quarter * kChunks + c;
                     if ((uint32_t)u % S != rank) continue;
                     uint32_t v[32];
@@ -449,7 +469,7 @@ inline int gemm_resident(int dev, int S, size_t smem) {
     }
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(1, 1, 1024);
-    q.blockDim = dim3(kGemmThreads);
+    q.blockDim = dim3(gemm_threads<FMT>());
     q.dynamicSmemBytes = smem;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -541,7 +561,7 @@ inline int launch_gemm_bn(const uint8_t *dT, int64_t ldp, float alpha, const uin
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((N + kGemmRows - 1) / kGemmRows), (unsigned)((M + BN - 1) / BN),
                        (unsigned)S);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(gemm_threads<FMT>());
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
