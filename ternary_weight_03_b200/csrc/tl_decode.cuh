@@ -1382,10 +1382,15 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     }
     // Items are handed out in table order.  Without dependencies between
     // layers, the costliest items go first, so the last ones handed out (the
-    // launch's tail) are the cheapest.
+    // launch's tail) are the cheapest.  A part of a split tile also counts
+    // the finish its tile may need (one round of loads per token and per
+    // four parts, about a stage each), so split tiles finish early.
     if (!sc.chained)
         std::stable_sort(items->begin(), items->end(), [](const DkItemRec &x, const DkItemRec &y) {
-            return (x.s1 - x.s0) * dk_stage_cost(x.M) > (y.s1 - y.s0) * dk_stage_cost(y.M);
+            auto cost = [](const DkItemRec &r) {
+                return (r.s1 - r.s0) * dk_stage_cost(r.M) + (r.parts > 1 ? r.M * ((r.parts + 3) / 4) : 0);
+            };
+            return cost(x) > cost(y);
         });
     return sc;
 }
