@@ -576,9 +576,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
     if (warp != 0) {
         // ---- every warp but the producer: convert activations, one unit at a time ----
         pdl_wait();  // X may be written by the preceding grid; Y may still be in use
-        // unit u goes to warp u mod (all converting warps of the grid)
+        // unit u goes to CTA u mod gridDim.x, so that every CTA converts a few
+        // units at once (one per warp) rather than a few CTAs many; within a
+        // CTA the stagers come last, as they convert the CTA's first item next
         constexpr int kConv = kDkWarps - 1;
-        for (int u = (int)blockIdx.x * kConv + warp - 1; u < a.total_units;
+        const int crank = warp > kDkStagers ? warp - 1 - kDkStagers : kConv - kDkStagers + warp - 1;
+        for (int u = crank * (int)gridDim.x + (int)blockIdx.x; u < a.total_units;
              u += (int)gridDim.x * kConv) {
             const DkUnitRec U = dk_load_rec<DkUnitRec, 3>(a.units, u);
             const int valid = min(U.K - U.stage * kDkStageTrits, kDkStageTrits);
