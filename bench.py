@@ -584,7 +584,7 @@ def time_ternarise(dev, stream, pk):
     return res
 
 
-def secondary(dev, stream, quick: bool):
+def secondary(dev, stream):
     """1.6-bit sweep (p0 = 1/3), batched GEMM (both formats), the 30-layer
     decode step, the device ternariser, the cold 1024 x 1024 single call and
     the sweep as separate per-layer calls."""
@@ -753,7 +753,7 @@ def run_gpu(args):
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if not args.no_secondary:
         try:  # context lines: an error there is recorded, the headline line still prints
-            line["secondary"] = secondary(dev, stream, quick=True)
+            line["secondary"] = secondary(dev, stream)
         except Exception as e:  # noqa: BLE001
             line["secondary"] = {"error": f"{type(e).__name__}: {e}"}
     if rank == 0:
