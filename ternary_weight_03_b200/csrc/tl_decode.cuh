@@ -1306,9 +1306,21 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows) *
                  dk_stage_cost(in[l].M);
     const int cost = dk_item_cost(total);
+    bool chained = false;
+    for (int l = 0; l < count; ++l) chained = chained || in[l].reads_earlier;
     // fp16-engine items stay at 8 stages or more: their epilogue (M outputs
-    // per row) must keep up with the consumers
+    // per row) must keep up with the consumers.  In a batch with chained
+    // layers, layers run one after another, so a layer's items are sized to
+    // spread it over about one CTA per SM instead (at most 8 parts per tile
+    // for the integer engine, 2 for the fp16 engine, whose final sums of
+    // split tiles cost more).
     auto target_of = [&](const DkHostLayer &h) {
+        if (chained) {
+            const int64_t units = (int64_t)stages_of(h) * ((h.N + kDkRows - 1) / kDkRows);
+            const int t = (int)((units + kDkRefSms - 1) / kDkRefSms);
+            const int min_t = (stages_of(h) + (h.M > kDkImmaMaxM ? 1 : 7)) / (h.M > kDkImmaMaxM ? 2 : 8);
+            return t > min_t ? t : (min_t > 0 ? min_t : 1);
+        }
         const int t = cost / dk_stage_cost(h.M);
         return h.M > kDkImmaMaxM && t < 8 ? 8 : t;
     };

@@ -135,17 +135,25 @@ def _ws2_expected(layers):
     (256-row tile x K-part of 2..16 stages of 512 trits), a 48-byte record per
     conversion unit (stage x token of a layer that reads no earlier output), a
     u32 per layer and per tile, 8-byte partials of split tiles, and the
-    converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage)."""
+    converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage).
+    With a chained layer in the batch, a layer's items are sized to spread it
+    over about 148 CTAs (at most 8 parts per tile, 2 for M > 2)."""
     items = units = tiles = slots = staged = 0
     stg = lambda d: -(-(-(-d["K"] // 4)) // 128)
     cm = lambda d: 1 if d["M"] <= 2 else 2  # relative cost of a stage
     total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
     cost = min(16, max(4, total // (4 * 148)))  # cost per item
+    chained = any(d.get("flags", 0) for d in layers)
     for d in layers:
         stages = stg(d)
-        target = max(1, cost // cm(d))
-        if d["M"] > 2:
-            target = max(target, 8)
+        if chained:
+            target = -(-stages * -(-d["N"] // 256) // 148)
+            min_t = -(-stages // (2 if d["M"] > 2 else 8))
+            target = max(target, min_t, 1)
+        else:
+            target = max(1, cost // cm(d))
+            if d["M"] > 2:
+                target = max(target, 8)
         parts = max(1, min(stages, (stages + target // 2) // target))
         t = -(-d["N"] // 256)
         items += t * parts
@@ -168,7 +176,9 @@ def test_batch_workspace_size(L):
     cases = [[dict(base, N=1000, K=2048)], [dict(base, N=4096, K=14336)],
              [dict(base, N=4096, K=14336, M=8)], [dict(base, N=4096, K=14336, M=2)],
              [dict(base, N=130, K=700, M=3), dict(base, N=77, K=5000, M=1, flags=1)],
-             [dict(base, N=14336, K=4096)] * 12, [dict(base, N=3072, K=8192, M=8)] * 80]
+             [dict(base, N=14336, K=4096)] * 12, [dict(base, N=3072, K=8192, M=8)] * 80,
+             [dict(base, N=3072, K=3072), dict(base, N=8192, K=3072, flags=1),
+              dict(base, N=3072, K=8192, flags=1), dict(base, N=3072, K=8192, M=8, flags=1)]]
     for ls in cases:
         arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16, ldx=d["K"] +
                             (-d["K"]) % 8, ldy=d["N"] + (-d["N"]) % 8) for d in ls])
