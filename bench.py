@@ -455,7 +455,11 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     own seeded activation vector(s), run as ONE tl_gemv_batch_run per step
     (graph-captured, programmatic dependent launch).  "chained" reruns the
     2-bit M = 1 step with every layer flagged as reading the earlier layers'
-    outputs (a serial dependency per layer).  Returns GB/s of packed weights."""
+    outputs (a serial dependency per layer).  "fused" (2-bit) runs the step
+    as a decoder would: q, k and v on one shared X (converted once), gate
+    and up on another, writing the two halves of one buffer, and down
+    reading silu(gate) * up from it (TL_LAYER_SWIGLU_INPUT, a dependency on
+    the earlier layers).  Returns GB/s of packed weights."""
     import torch
     import synth
     import ternary_weight_03_b200 as tl
@@ -511,6 +515,35 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
                     "packed_bytes": total, "us_per_step": round(ms_step * 1e3, 2),
                     "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks()["hbm_gbs"], 4)}
                 del plan, ws
+            if fmt == 2:
+                # the fused step: per decoder layer q, k, v share X; gate and up
+                # share another X and fill [gate | up]; down reads silu(gate) * up
+                specs = []
+                for layer in range(30):
+                    base = 7 * layer
+                    xa, xo, xf = xs[base], xs[base + 3], xs[base + 4]
+                    gu = torch.empty((M, 2 * 8192), dtype=torch.float16, device=dev)
+                    for j in range(7):
+                        K, N, dP, alpha = dev_mats[base + j]
+                        if j < 3:
+                            specs.append((dP, alpha, xa, K, ys[base + j]))
+                        elif j == 3:
+                            specs.append((dP, alpha, xo, K, ys[base + j]))
+                        elif j < 6:
+                            half = gu[:, :8192] if j == 4 else gu[:, 8192:]
+                            specs.append((dP, alpha, xf, K, half))
+                        else:
+                            specs.append((dP, alpha, gu, K, ys[base + j],
+                                          tl.LAYER_READS_EARLIER | tl.LAYER_SWIGLU_INPUT))
+                layers = tl.make_layers(fmt, specs)
+                ws = torch.zeros(tl.gemv_batch_bytes(fmt, layers), dtype=torch.uint8, device=dev)
+                plan = tl.gemv_batch_plan(fmt, layers, ws)
+                ms_step = timed(plan)
+                gbs = total / (ms_step * 1e-3) / 1e9
+                out[f"fmt{fmt}_M{M}_fused"] = {
+                    "packed_bytes": total, "us_per_step": round(ms_step * 1e3, 2),
+                    "GB/s": round(gbs, 1), "frac_hbm": round(gbs / peaks()["hbm_gbs"], 4)}
+                del plan, ws, specs
             del xs, ys
         del dev_mats
         torch.cuda.empty_cache()

@@ -136,6 +136,7 @@ int tl_gemv_ex(int fmt, const uint8_t *dT, int64_t ldp, float alpha, const uint1
 
 #define TL_GEMV_BATCH_MAX 4096    /* layers per batch */
 #define TL_LAYER_READS_EARLIER 1u /* tl_gemv_layer.flags, see tl_gemv_batch_plan */
+#define TL_LAYER_SWIGLU_INPUT 2u  /* tl_gemv_layer.flags, see tl_gemv_batch_plan */
 
 /* One layer of a batch: the arguments of tl_gemv for that layer. */
 typedef struct tl_gemv_layer {
@@ -148,7 +149,7 @@ typedef struct tl_gemv_layer {
     int64_t ldy;
     int M;               /* 1 .. TL_GEMV_MAX_M */
     int64_t N, K;
-    unsigned int flags;  /* 0 or TL_LAYER_READS_EARLIER */
+    unsigned int flags;  /* 0, TL_LAYER_READS_EARLIER, or that | TL_LAYER_SWIGLU_INPUT */
 } tl_gemv_layer;
 
 /* A planned batch: filled by tl_gemv_batch_plan, read by tl_gemv_batch_run.
@@ -156,7 +157,8 @@ typedef struct tl_gemv_layer {
 typedef struct tl_gemv_plan {
     int fmt, count, max_m, total_items, total_tiles;
     int total_units;  /* activation conversion units of the launch */
-    int chained;      /* 1 if some layer has TL_LAYER_READS_EARLIER */
+    int chained;      /* 1 if some layer has TL_LAYER_READS_EARLIER, 2 if one
+                         also has TL_LAYER_SWIGLU_INPUT, else 0 */
     void *dWorkspace;
     size_t workspace_bytes;
     uint64_t generation; /* 0, or the static plan's number (tl_gemv_batch_plan_static) */
@@ -189,8 +191,22 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
  * 0) reads its X only after every earlier layer of the batch has stored its
  * Y, so it may consume their outputs (a chain of layers); without the flag,
  * X must not be written by any layer of the batch.  No Y may overlap another
- * layer's Y, X or T.  Errors: TL_ERR_INVALID_ARG (bad layer, count or
- * workspace too small), TL_ERR_ALIGN, TL_ERR_CUDA. */
+ * layer's Y, X or T.
+ * SwiGLU input (2-bit only; TL_LAYER_SWIGLU_INPUT together with
+ * TL_LAYER_READS_EARLIER): row m of dX holds a gated unit's two inputs, the
+ * gate values g in elements [0, K) and the up values u in [K, 2K) (typically
+ * the outputs of two earlier layers writing the halves of one buffer), and
+ * the layer's input is x_k = fp16_rn(silu(g_k) * u_k), silu(g) = g / (1 +
+ * exp(-g)), evaluated in fp32 -- the gated feed-forward unit of a LLaMA-style
+ * decoder fused into its down projection, so the product never goes to
+ * memory.  Needs ldx >= 2 K and K % 8 == 0 (else TL_ERR_INVALID_ARG /
+ * TL_ERR_ALIGN); the 1.6-bit batch returns TL_ERR_UNSUPPORTED.
+ * Independent layers with the same X (pointer, ldx, K and M; no
+ * TL_LAYER_READS_EARLIER), such as the Q, K and V projections of one token
+ * batch, share one conversion of X: it is staged once per launch, and each
+ * layer keeps its own alpha.
+ * Errors: TL_ERR_INVALID_ARG (bad layer, count or workspace too small),
+ * TL_ERR_ALIGN, TL_ERR_UNSUPPORTED, TL_ERR_CUDA. */
 int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dWorkspace,
                        size_t workspace_bytes, tl_gemv_plan *plan);
 

@@ -29,6 +29,7 @@ STATUS = {0: "TL_OK", 1: "TL_ERR_INVALID_ARG", 2: "TL_ERR_BAD_TRIT", 3: "TL_ERR_
 
 GEMV_BATCH_MAX = 4096
 LAYER_READS_EARLIER = 1
+LAYER_SWIGLU_INPUT = 2
 
 
 class Layer(ctypes.Structure):

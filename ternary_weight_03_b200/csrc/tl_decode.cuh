@@ -117,13 +117,15 @@ struct DkItemRec {
     const uint8_t *B;  // converted operands of the layer ([meta][B] per stage), or null
     int64_t part_off;  // first 8-byte partial slot of the item's layer
     float alpha;
-    int layer;         // index of the layer's tensor map
+    int layer;         // low 16 bits: the layer (its tensor map); high 16 bits: the
+                       // layer whose conversion of X it uses (its ready counter)
     int tile, part, s0, s1;
     int M, K, N, ldx, ldy;
     int parts;         // K-parts per tile of the layer
     int tile_begin;    // global index of the layer's first tile
     int wait_tiles;    // tiles that must be final before X is read (0: none)
-    int need;          // conversion units of the layer (stages x M)
+    int need;          // conversion units of X (stages x M); chained layers: 1 if X
+                       // holds [gate | up] halves (SwiGLU input), else 0
     int bstride;       // bytes per stage of B (64 + dk_stage_b(M))
 };
 static_assert(sizeof(DkItemRec) == 96, "item record is six 16-byte loads");
@@ -174,7 +176,7 @@ struct DkArgs {
     int total_items;
     int total_units;
     int maxM;
-    int chained;  // some layer reads an earlier layer's output
+    int chained;  // 1: some layer reads an earlier layer's output; 2: and one has a SwiGLU input
     int drop_arrive;  // failure-detection hook (debug library only), else 0
 };
 
@@ -187,7 +189,7 @@ struct DkQEntry {
     int tile, part, s0, s1, M, K, N, ldx, ldy, parts, tile_begin;
     int pre;      // 1: converted operands arrive with the weights; 0: a stager converts X
     int chained;  // X is written by earlier layers of this launch
-    int pad_;
+    int swiglu;   // X rows hold [gate | up]; the input is silu(gate) * up
 };
 
 struct DkLayout {
@@ -353,18 +355,45 @@ __device__ __forceinline__ void dk_read_word(const uint16_t *src, int w, int val
     }
 }
 
+// The same for a SwiGLU input: element e of the word is
+// fp16_rn(silu(g_e) * u_e) in fp32, g from src and u from up = src + K (the
+// row's second half); zero at e >= valid.
+__device__ __forceinline__ void dk_read_word_glu(const uint16_t *src, const uint16_t *up, int w,
+                                                 int valid, uint32_t (&r)[8]) {
+    uint32_t g[8], u[8];
+    dk_read_word(src, w, valid, g);
+    dk_read_word(up, w, valid, u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 gf = __half22float2(*reinterpret_cast<const __half2 *>(&g[i]));
+        const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&u[i]));
+        const float a = gf.x / (1.0f + expf(-gf.x)) * uf.x;
+        const float b = gf.y / (1.0f + expf(-gf.y)) * uf.y;
+        const __half2 h = __floats2half2_rn(a, b);
+        r[i] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+}
+// One word of a stage's activations: plain, or the SwiGLU product (up != null).
+__device__ __forceinline__ void dk_load_word(const uint16_t *src, const uint16_t *up, int w,
+                                             int valid, uint32_t (&r)[8]) {
+    if (up)
+        dk_read_word_glu(src, up, w, valid, r);
+    else
+        dk_read_word(src, w, valid, r);
+}
+
 // One warp converts one stage of token m for the integer engine: z = x 2^24 +
 // 2^40 as six u8 planes, each 16-byte block the 4x4 transpose of a word's
 // elements (byte 4j + b = element 4b + j), the ones column (m == 0), and
 // Q = sum x 2^24 into meta[m] (exact: the partial sums of binary16 values are
 // multiples of 2^-24 below 2^26, within a double's 53 bits).
-__device__ __forceinline__ void dk_conv_imma(const uint16_t *src, int valid, int m, int M,
-                                             uint8_t *dstB, uint8_t *meta, int lane) {
+__device__ __forceinline__ void dk_conv_imma(const uint16_t *src, const uint16_t *up, int valid,
+                                             int m, int M, uint8_t *dstB, uint8_t *meta, int lane) {
     const int ones = dk_ones_col(M);
     double qd = 0.0;
     for (int w = lane; w < kDkWords; w += 32) {
         uint32_t r[8];
-        dk_read_word(src, w, valid, r);
+        dk_load_word(src, up, w, valid, r);
         uint32_t lo[16], hi[16];
 #pragma unroll
         for (int e2 = 0; e2 < 16; e2 += 2) {
@@ -410,12 +439,12 @@ __device__ __forceinline__ void dk_conv_imma(const uint16_t *src, int valid, int
 // One warp converts one stage of token m for the fp16 engine: per word and
 // digit position j the pairs (x_j, x_{8+j}) and (x_{4+j}, x_{12+j}), and
 // sum_k x into meta[m] (fp32).
-__device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, int valid, int m, int Mp,
-                                             uint8_t *dstB, uint8_t *meta, int lane) {
+__device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, const uint16_t *up, int valid,
+                                             int m, int Mp, uint8_t *dstB, uint8_t *meta, int lane) {
     float sx = 0.f;
     for (int w = lane; w < kDkWords; w += 32) {
         uint32_t r[8];
-        dk_read_word(src, w, valid, r);
+        dk_load_word(src, up, w, valid, r);
         uint32_t b[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -532,6 +561,9 @@ __device__ __noinline__ void dk_finalize(const int64_t *base, int cnt, int parts
     }
 }
 
+// kGlu: the batch has SwiGLU-input layers (a separate instantiation, so that
+// the conversion's fp32 silu code is not part of every other batch's kernel).
+template <bool kGlu>
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
     extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
     const DkLayout lay(a.maxM);
@@ -587,9 +619,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             const int valid = min(U.K - U.stage * kDkStageTrits, kDkStageTrits);
             const uint16_t *src = U.X + (int64_t)U.m * U.ldx + (int64_t)U.stage * kDkStageTrits;
             if (U.M <= kDkImmaMaxM)
-                dk_conv_imma(src, valid, U.m, U.M, U.dst + kDkMetaBytes, U.dst, lane);
+                dk_conv_imma(src, nullptr, valid, U.m, U.M, U.dst + kDkMetaBytes, U.dst, lane);
             else
-                dk_conv_hmma(src, valid, U.m, U.M + (U.M & 1), U.dst + kDkMetaBytes, U.dst, lane);
+                dk_conv_hmma(src, nullptr, valid, U.m, U.M + (U.M & 1), U.dst + kDkMetaBytes, U.dst,
+                             lane);
             // the converted unit is read by bulk copies of other CTAs
             dk_fence_proxy_global();
             __threadfence();
@@ -653,13 +686,14 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     e.tile_begin = R.tile_begin;
                     e.pre = pre ? 1 : 0;
                     e.chained = R.wait_tiles > 0 ? 1 : 0;
+                    e.swiglu = R.wait_tiles > 0 && (R.need & 1) ? 1 : 0;
                 }
                 queue[q] = e;
                 mbar_arrive(&qfull[q]);
             }
             ++qi;
             if (!valid) break;
-            const CUtensorMap *tmap = a.maps + R.layer;
+            const CUtensorMap *tmap = a.maps + (R.layer & 0xFFFF);
             const int n0 = R.tile * kDkRows;
             // bytes of a stage besides the weights: the converted operands
             auto extra = [&](int) -> uint32_t { return pre ? (uint32_t)R.bstride : 0u; };
@@ -677,7 +711,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 bool good = true;
                 if (pre) {
                     if (!all_ready) {
-                        good = dk_wait_count(&a.ready[R.layer], (uint32_t)R.need,
+                        good = dk_wait_count(&a.ready[R.layer >> 16], (uint32_t)R.need,
                                              &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
                         fenced = false;
                     }
@@ -767,7 +801,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             item = next;
             R = NR;
             next = next < a.total_items ? __shfl_sync(0xffffffffu, nx2, 0) : a.total_items;
-            if (item < a.total_items && lane == 0) tma_prefetch_desc(a.maps + R.layer);
+            if (item < a.total_items && lane == 0) tma_prefetch_desc(a.maps + (R.layer & 0xFFFF));
         }
         if (!waited) pdl_wait();
         // the CTA may not exit with copies still landing in its shared memory
@@ -818,10 +852,11 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 uint8_t *dst = sslot + slot * lay.slot_b;
                 for (int m = 0; m < M; ++m) {
                     const uint16_t *src = e.X + (int64_t)m * e.ldx + (int64_t)s * kDkStageTrits;
+                    const uint16_t *up = kGlu && e.swiglu ? src + K : nullptr;  // [gate | up] rows
                     if (M <= kDkImmaMaxM)
-                        dk_conv_imma(src, valid, m, M, dst + kDkMetaBytes, dst, lane);
+                        dk_conv_imma(src, up, valid, m, M, dst + kDkMetaBytes, dst, lane);
                     else
-                        dk_conv_hmma(src, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
+                        dk_conv_hmma(src, up, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
                 }
 #ifdef TL_DEBUG_HOOKS
                 // the hook: CTA 0's first stage converted here is never published
@@ -1282,6 +1317,7 @@ struct DkHostLayer {
     float alpha;
     int M, N, K;
     bool reads_earlier;
+    bool swiglu;  // X rows hold [gate | up] (only with reads_earlier)
 };
 
 struct DkSchedule {
@@ -1324,6 +1360,20 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         const int t = cost / dk_stage_cost(h.M);
         return h.M > kDkImmaMaxM && t < 8 ? 8 : t;
     };
+    // An independent layer whose X (pointer, stride, K, M) is an earlier
+    // independent layer's uses that layer's conversion (Q, K and V of one
+    // token batch convert X once); src[l] is the layer that converts.
+    std::vector<int> src(count);
+    for (int l = 0; l < count; ++l) {
+        src[l] = l;
+        if (in[l].reads_earlier) continue;
+        for (int j = 0; j < l; ++j)
+            if (src[j] == j && !in[j].reads_earlier && in[j].X == in[l].X &&
+                in[j].ldx == in[l].ldx && in[j].K == in[l].K && in[j].M == in[l].M) {
+                src[l] = j;
+                break;
+            }
+    }
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
         const int stages = stages_of(h);
@@ -1332,8 +1382,9 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         sc.total_items += tiles * parts;
         sc.total_tiles += tiles;
         if (h.reads_earlier) {
-            sc.chained = 1;
-        } else {
+            if (sc.chained == 0) sc.chained = 1;
+            if (h.swiglu) sc.chained = 2;
+        } else if (src[l] == l) {
             sc.total_units += stages * h.M;
             sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(h.M));
         }
@@ -1345,13 +1396,16 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     if (!items || !units) return sc;
     int64_t slots = 0, staged = 0;
     int tile_begin = 0;
+    std::vector<uint8_t *> Bs(count, nullptr);  // each layer's converted X
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
         const int stages = stages_of(h);
         const int parts = dk_parts(stages, target_of(h));
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         const int bstride = kDkMetaBytes + (int)dk_stage_b(h.M);
-        uint8_t *B = h.reads_earlier ? nullptr : ws + wl.staged + staged;
+        const bool converts = !h.reads_earlier && src[l] == l;
+        uint8_t *B = h.reads_earlier ? nullptr : (converts ? ws + wl.staged + staged : Bs[src[l]]);
+        Bs[l] = B;
         for (int t = 0; t < tiles; ++t)
             for (int q = 0; q < parts; ++q) {
                 DkItemRec r{};
@@ -1360,7 +1414,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
                 r.B = B;
                 r.part_off = slots;
                 r.alpha = h.alpha;
-                r.layer = l;
+                r.layer = l | (src[l] << 16);
                 r.tile = t;
                 r.part = q;
                 r.s0 = (int)((int64_t)stages * q / parts);
@@ -1373,11 +1427,11 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
                 r.parts = parts;
                 r.tile_begin = tile_begin;
                 r.wait_tiles = h.reads_earlier ? tile_begin : 0;
-                r.need = stages * h.M;
+                r.need = h.reads_earlier ? (h.swiglu ? 1 : 0) : stages * h.M;
                 r.bstride = bstride;
                 items->push_back(r);
             }
-        if (B)
+        if (converts)
             for (int s = 0; s < stages; ++s)
                 for (int m = 0; m < h.M; ++m) {
                     DkUnitRec u{};
@@ -1392,7 +1446,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
                     units->push_back(u);
                 }
         if (parts > 1) slots += (int64_t)tiles * parts * kDkRows * h.M;
-        if (B) staged += (int64_t)stages * bstride;
+        if (converts) staged += (int64_t)stages * bstride;
         tile_begin += tiles;
     }
     // Items are handed out in table order.  Without dependencies between
@@ -1464,8 +1518,11 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
             const uint32_t t = DkLayout(m).total;
             most = t > most ? t : most;
         }
-        attr_err[dev] = cudaFuncSetAttribute(decode2_kernel,
+        attr_err[dev] = cudaFuncSetAttribute(decode2_kernel<false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+        if (attr_err[dev] == cudaSuccess)
+            attr_err[dev] = cudaFuncSetAttribute(
+                decode2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
     });
     if (attr_err[dev] != cudaSuccess) {
         *last_cuda_error = (int)attr_err[dev];
@@ -1481,7 +1538,8 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = pdl ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, decode2_kernel, a);
+    e = a.chained == 2 ? cudaLaunchKernelEx(&cfg, decode2_kernel<true>, a)
+                       : cudaLaunchKernelEx(&cfg, decode2_kernel<false>, a);
     if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;

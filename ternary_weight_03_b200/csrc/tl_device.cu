@@ -101,16 +101,25 @@ int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::GpHostLay
     for (int l = 0; l < count; ++l) {
         const tl_gemv_layer &a = layers[l];
         if (a.M < 1 || a.M > TL_GEMV_MAX_M) return TL_ERR_INVALID_ARG;
-        if (a.flags & ~(unsigned int)TL_LAYER_READS_EARLIER) return TL_ERR_INVALID_ARG;
+        constexpr unsigned int kFlags = TL_LAYER_READS_EARLIER | TL_LAYER_SWIGLU_INPUT;
+        if (a.flags & ~kFlags) return TL_ERR_INVALID_ARG;
         if (l == 0 && (a.flags & TL_LAYER_READS_EARLIER)) return TL_ERR_INVALID_ARG;
+        const bool swiglu = (a.flags & TL_LAYER_SWIGLU_INPUT) != 0;
+        if (swiglu && !(a.flags & TL_LAYER_READS_EARLIER)) return TL_ERR_INVALID_ARG;
         int rc = check_layer_args(fmt, a.dT, a.ldp, a.dX, a.ldx, a.dY, a.ldy, a.N, a.K);
         if (rc != TL_OK) return rc;
+        if (swiglu) {
+            // X rows hold [gate | up]: 2K elements, the up half 16-byte aligned
+            if (a.ldx < 2 * a.K) return TL_ERR_INVALID_ARG;
+            if (a.K % 8 != 0) return TL_ERR_ALIGN;
+            if (fmt != TL_FMT_2BIT) return TL_ERR_UNSUPPORTED;
+        }
         if (a.ldx > INT32_MAX || a.ldy > INT32_MAX) return TL_ERR_INVALID_ARG;
         const int64_t groups = (tl_packed_row_bytes(fmt, a.K) + 63) / 64;
         items += ((a.N + tlk::kGpRows - 1) / tlk::kGpRows) * groups;  // upper bound
         if (items > INT32_MAX / 2) return TL_ERR_INVALID_ARG;
         out[l] = tlk::GpHostLayer{a.dT, a.dX, a.dY, a.ldp, a.ldx, a.ldy, a.alpha, a.M, (int)a.N,
-                                  (int)a.K, (a.flags & TL_LAYER_READS_EARLIER) != 0};
+                                  (int)a.K, (a.flags & TL_LAYER_READS_EARLIER) != 0, swiglu};
     }
     return TL_OK;
 }
@@ -120,7 +129,8 @@ std::vector<tlk::DkHostLayer> dk_layers(const std::vector<tlk::GpHostLayer> &h) 
     std::vector<tlk::DkHostLayer> out(h.size());
     for (size_t l = 0; l < h.size(); ++l)
         out[l] = tlk::DkHostLayer{h[l].T, h[l].X, h[l].Y, h[l].ldp, h[l].ldx, h[l].ldy,
-                                  h[l].alpha, h[l].M, h[l].N, h[l].K, h[l].reads_earlier};
+                                  h[l].alpha, h[l].M, h[l].N, h[l].K, h[l].reads_earlier,
+                                  h[l].swiglu};
     return out;
 }
 
@@ -337,7 +347,7 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
     if (plan->fmt != TL_FMT_2BIT && plan->fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
     if (plan->count < 1 || plan->count > TL_GEMV_BATCH_MAX || plan->max_m < 1 ||
         plan->max_m > TL_GEMV_MAX_M || plan->total_items < 1 || plan->total_tiles < 1 ||
-        plan->total_units < 0 || (plan->chained != 0 && plan->chained != 1))
+        plan->total_units < 0 || plan->chained < 0 || plan->chained > 2)
         return TL_ERR_INVALID_ARG;
     const DeviceInfo *dev = device_info();
     if (!dev) return TL_ERR_CUDA;

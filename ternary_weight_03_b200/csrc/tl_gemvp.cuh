@@ -687,6 +687,7 @@ struct GpHostLayer {
     float alpha;
     int M, N, K;
     bool reads_earlier;
+    bool swiglu = false;  // X holds gate and up halves (2-bit batch only)
 };
 
 struct GpSchedule {

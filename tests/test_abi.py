@@ -137,13 +137,16 @@ def _ws2_expected(layers):
     u32 per layer and per tile, 8-byte partials of split tiles, and the
     converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage).
     With a chained layer in the batch, a layer's items are sized to spread it
-    over about 148 CTAs (at most 8 parts per tile, 2 for M > 2)."""
+    over about 148 CTAs (at most 8 parts per tile, 2 for M > 2).  Independent
+    layers with the same X (pointer, ldx, K, M) share the first one's
+    conversion (no units or converted activations of their own)."""
     items = units = tiles = slots = staged = 0
     stg = lambda d: -(-(-(-d["K"] // 4)) // 128)
     cm = lambda d: 1 if d["M"] <= 2 else 2  # relative cost of a stage
     total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
     cost = min(16, max(4, total // (4 * 148)))  # cost per item
     chained = any(d.get("flags", 0) for d in layers)
+    seen = set()
     for d in layers:
         stages = stg(d)
         if chained:
@@ -158,7 +161,9 @@ def _ws2_expected(layers):
         t = -(-d["N"] // 256)
         items += t * parts
         tiles += t
-        if not d.get("flags", 0):
+        key = (d.get("dX", A), d.get("ldx", d["K"] + (-d["K"]) % 8), d["K"], d["M"])
+        if not d.get("flags", 0) and key not in seen:
+            seen.add(key)
             units += stages * d["M"]
             b = 4096 if d["M"] == 1 else (8192 if d["M"] == 2 else 1024 * (d["M"] + d["M"] % 2))
             staged += stages * (64 + b)
@@ -178,10 +183,16 @@ def test_batch_workspace_size(L):
              [dict(base, N=130, K=700, M=3), dict(base, N=77, K=5000, M=1, flags=1)],
              [dict(base, N=14336, K=4096)] * 12, [dict(base, N=3072, K=8192, M=8)] * 80,
              [dict(base, N=3072, K=3072), dict(base, N=8192, K=3072, flags=1),
-              dict(base, N=3072, K=8192, flags=1), dict(base, N=3072, K=8192, M=8, flags=1)]]
+              dict(base, N=3072, K=8192, flags=1), dict(base, N=3072, K=8192, M=8, flags=1)],
+             # Q, K, V on one X (one conversion), O on its own X, gate and up on a
+             # third X, the down projection reading silu(gate) * up
+             [dict(base, N=3072, K=3072, M=2)] * 3 + [dict(base, N=3072, K=3072, M=2, dX=A + 65536)]
+             + [dict(base, N=8192, K=3072, M=2, dX=A + 131072)] * 2
+             + [dict(base, N=3072, K=8192, M=2, flags=3, ldx=16384)]]
     for ls in cases:
-        arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16, ldx=d["K"] +
-                            (-d["K"]) % 8, ldy=d["N"] + (-d["N"]) % 8) for d in ls])
+        arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16,
+                            ldx=d.get("ldx", d["K"] + (-d["K"]) % 8),
+                            ldy=d["N"] + (-d["N"]) % 8) for d in ls])
         rc, n = _ws(L, 2, arr)
         assert rc == 0 and n == _ws2_expected(ls), (ls, n)
     # 1.6-bit: table (one 88-byte entry + one 128-byte TMA descriptor per layer),
@@ -202,6 +213,22 @@ def test_batch_argument_rules(L, spec, count, rc):
     plan = tl.Plan()
     assert L.tl_gemv_batch_bytes(2, count, arr, ctypes.byref(n)) == rc
     assert L.tl_gemv_batch_plan(2, count, arr, A, 1 << 20, ctypes.byref(plan)) == rc
+
+
+@pytest.mark.parametrize("fmt,second,rc", [
+    (2, dict(flags=3, ldx=2048), 0),                 # [gate | up] rows of 2K elements
+    (2, dict(flags=2, ldx=2048), 1),                 # SwiGLU input needs READS_EARLIER
+    (2, dict(flags=3, ldx=1024), 1),                 # rows shorter than 2K
+    (2, dict(flags=3, K=1020, ldx=2048, ldp=256), 4),  # up half not 16-byte aligned
+    (2, dict(flags=4), 1),                           # unknown flag
+    (16, dict(flags=3, ldx=2048), 7),                # 1.6-bit batch: unsupported
+])
+def test_swiglu_input_rules(L, fmt, second, rc):
+    import ctypes
+    first = dict(ldp=256 if fmt == 2 else 208)
+    arr = _layers([first, dict(first, **second)])
+    n = ctypes.c_size_t(0)
+    assert L.tl_gemv_batch_bytes(fmt, 2, arr, ctypes.byref(n)) == rc
 
 
 def test_batch_plan_and_run_rules(L):

@@ -319,3 +319,89 @@ def test_decode_step_210_layers_sampled(fmt, M):
         ref = o.linear_at(T, X, sp[1], ms, ns)
         tol = oracle.tolerance(ref, X[ms], sp[1])
         assert (np.abs(Y[ms, ns] - ref) <= tol).all(), f"layer seed {seed}"
+
+
+def _silu_glu(gu, F):
+    """silu(g) * u in double from a [gate | up] row block of fp16 values."""
+    g = gu[:, :F].astype(np.float64)
+    u = gu[:, F:2 * F].astype(np.float64)
+    return g / (1.0 + np.exp(-g)) * u
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 8])
+def test_swiglu_down_projection(M):
+    """Gate and up projections write the two halves of one buffer; the down
+    projection reads it with TL_LAYER_SWIGLU_INPUT, its input formed on chip
+    as fp16(silu(g) * u).  Checked layer by layer against the oracle: gate
+    and up as plain layers, the down projection against the oracle applied to
+    silu(g) * u computed here in double from the stored gate and up outputs
+    and rounded to binary16, the bound adding alpha * sum_k ulp16(x_k) for the
+    one-ulp freedom of that rounding.  An independent layer sits between."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    H, F, H2 = 3000, 1000, 700
+    X0 = synth.activations(80 + M, M, H)
+    Tg, Tu = synth.trits(81, F, H), synth.trits(82, F, H)
+    Tx = synth.trits(84, 500, H)
+    Td = synth.trits(83, H2, F)
+    ag, au, ax, ad = 0.021, 0.033, 0.04, 0.017
+    dX0 = torch.from_numpy(X0).cuda()
+    GU = torch.full((M, 2 * F), float("nan"), dtype=torch.float16, device="cuda")
+    Yx = torch.full((M, 504), float("nan"), dtype=torch.float16, device="cuda")
+    Yd = torch.full((M, H2 + (-H2) % 8), float("nan"), dtype=torch.float16, device="cuda")
+    pk = lambda T: torch.from_numpy(tl.pack(2, T)).cuda()
+    specs = [(pk(Tg), ag, dX0, H, GU[:, :F]), (pk(Tu), au, dX0, H, GU[:, F:]),
+             (pk(Tx), ax, dX0, H, Yx),
+             (pk(Td), ad, GU, F, Yd, tl.LAYER_READS_EARLIER | tl.LAYER_SWIGLU_INPUT)]
+    layers = tl.make_layers(2, specs)
+    plan, ws = _plan(2, layers)
+    outs = []
+    for _ in range(2):
+        Yd.fill_(float("nan"))
+        tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+        assert tl.device_status() == 0
+        outs.append(Yd.cpu().numpy().view(np.uint16).copy())
+    assert np.array_equal(outs[0], outs[1]), "not deterministic"
+    o = oracle.get()
+    gu = GU.cpu().numpy()
+    for T, a, Y in ((Tg, ag, gu[:, :F]), (Tu, au, gu[:, F:]), (Tx, ax, Yx[:, :500].cpu().numpy())):
+        ref = o.linear(T, X0, a, nthreads=8)
+        assert (np.abs(Y.astype(np.float64) - ref) <= oracle.tolerance(ref, X0, a)).all()
+    x = _silu_glu(gu, F).astype(np.float16)  # the down projection's input, rounded once
+    ref = o.linear(Td, x, ad, nthreads=8)
+    ulp = np.spacing(np.abs(x)).astype(np.float64)
+    tol = oracle.tolerance(ref, x, ad) + abs(ad) * ulp.sum(axis=1)[:, None]
+    got = Yd[:, :H2].float().cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref) <= tol).all(), f"{int((np.abs(got - ref) > tol).sum())} outside"
+    assert np.isnan(Yd[:, H2:].float().cpu().numpy()).all(), "wrote past column N"
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_layers_sharing_x(M):
+    """Q, K and V on one X (one conversion of X, three alphas), O on another
+    X, and two layers on a third: each layer against the oracle, and the
+    batch needs less workspace than the same layers on distinct X copies."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    K = 2000
+    Xa, Xb, Xc = (synth.activations(90 + i + M, M, K) for i in range(3))
+    dXa, dXb, dXc = (torch.from_numpy(v).cuda() for v in (Xa, Xb, Xc))
+    shapes = [(700, 0.02, 0), (300, 0.03, 0), (300, 0.045, 0), (700, 0.011, 1), (1200, 0.05, 2),
+              (1200, 0.013, 2)]
+    xs = [(Xa, dXa), (Xb, dXb), (Xc, dXc)]
+    cases, specs, specs_copy = [], [], []
+    for i, (N, a, xi) in enumerate(shapes):
+        T = synth.trits(95 + i, N, K)
+        dP = torch.from_numpy(tl.pack(2, T)).cuda()
+        dY = torch.full((M + 1, N + (-N) % 8), float("nan"), dtype=torch.float16, device="cuda")
+        specs.append((dP, a, xs[xi][1], K, dY[:M]))
+        specs_copy.append((dP, a, xs[xi][1].clone(), K, dY[:M]))
+        cases.append((T, xs[xi][0], a, dY, N))  # row M is a guard row
+    layers = tl.make_layers(2, specs)
+    shared_bytes = tl.gemv_batch_bytes(2, layers)
+    assert shared_bytes < tl.gemv_batch_bytes(2, tl.make_layers(2, specs_copy))
+    plan, ws = _plan(2, layers)
+    tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+    assert tl.device_status() == 0
+    for T, X, a, dY, N in cases:
+        _check_layer(T, X, a, dY, N, M)
