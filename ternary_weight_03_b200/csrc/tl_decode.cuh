@@ -92,7 +92,7 @@ constexpr uint32_t kDkSmemBudget = 232448u;             // 227 KB
 constexpr int kDkMetaBytes = 64;                        // per stage: per-token offsets, first
 
 // Workspace counters (u32 words of the 256-byte header).
-constexpr int kDkCtrFinal = 1;      // tiles whose outputs are stored
+constexpr int kDkCtrPrefix = 1;     // layers 0 .. prefix - 1 have all their outputs stored
 constexpr int kDkCtrDone = 2;       // CTAs that have finished
 constexpr int kDkCtrItems = 3;      // items handed out beyond the first 2 gridDim.x
 constexpr int kDkCtrUnitsDone = 5;  // CTAs whose conversion units are all written
@@ -123,7 +123,7 @@ struct DkItemRec {
     int M, K, N, ldx, ldy;
     int parts;         // K-parts per tile of the layer
     int tile_begin;    // global index of the layer's first tile
-    int wait_tiles;    // tiles that must be final before X is read (0: none)
+    int wait_tiles;    // 1: X is read once every earlier layer is complete (0: no wait)
     int need;          // conversion units of X (stages x M); chained layers: 1 if X
                        // holds [gate | up] halves (SwiGLU input), else 0
     int bstride;       // bytes per stage of B (64 + dk_stage_b(M))
@@ -144,7 +144,8 @@ static_assert(sizeof(DkUnitRec) == 48, "unit record is three 16-byte loads");
 //   maps    : count x CUtensorMap
 //   items   : total_items x DkItemRec
 //   units   : total_units x DkUnitRec
-//   ready   : count x u32, conversion units written per layer
+//   ready   : count x u32, conversion units written per layer; then count x u32,
+//             final tiles per layer; then count x u32, tiles per layer
 //   tiles   : total_tiles x u32, parts of each tile that have arrived
 //   partials: 8-byte partial sums of split tiles (int64 for M <= 2, double above)
 //   staged  : converted operands, per layer stages x (64 + dk_stage_b(M)) bytes
@@ -157,7 +158,7 @@ struct DkWsLayout {
         items = up(maps + (size_t)count * sizeof(CUtensorMap));
         units = up(items + (size_t)total_items * sizeof(DkItemRec));
         ready = up(units + (size_t)total_units * sizeof(DkUnitRec));
-        tiles = up(ready + (size_t)count * 4u);
+        tiles = up(ready + (size_t)count * 12u);
         partials = up(tiles + (size_t)total_tiles * 4u);
         staged = up(partials + (size_t)slots * 8u);
         total = up(staged + (size_t)staged_bytes);
@@ -170,6 +171,8 @@ struct DkArgs {
     const DkItemRec *items;
     const DkUnitRec *units;
     uint32_t *ready;
+    uint32_t *lfinal;        // final tiles per layer (batches with dependencies)
+    const uint32_t *ltiles;  // tiles per layer
     uint32_t *tile_ctr;
     int64_t *partials;
     int count;
@@ -190,6 +193,7 @@ struct DkQEntry {
     int pre;      // 1: converted operands arrive with the weights; 0: a stager converts X
     int chained;  // X is written by earlier layers of this launch
     int swiglu;   // X rows hold [gate | up]; the input is silu(gate) * up
+    int layer;    // the item's layer
 };
 
 struct DkLayout {
@@ -201,7 +205,7 @@ struct DkLayout {
         const uint32_t per_stage = (uint32_t)kDkWBytes + slot_b;
         const uint32_t fixed = nbufs * parts + kDkQueue * (uint32_t)sizeof(DkQEntry) +
                                8u * (3u * kDkMaxStages + 2u * kDkQueue + 2u * kDkMaxPartBufs) +
-                               16u + 1024u;  // a counter; alignment slack of the dynamic base
+                               16u + 4u * kDkQueue + 1024u;  // counter, ready words, base slack
         const uint32_t n = (kDkSmemBudget - fixed) / per_stage;
         ns = n > (uint32_t)kDkMaxStages ? (uint32_t)kDkMaxStages : n;  // >= 3 for maxM <= 8
         w_off = 0;
@@ -209,7 +213,7 @@ struct DkLayout {
         part_off = st_off + ns * slot_b;
         q_off = part_off + nbufs * parts;
         bar_off = (q_off + kDkQueue * (uint32_t)sizeof(DkQEntry) + 7u) & ~7u;
-        total = bar_off + 8u * (3u * ns + 2u * kDkQueue + 2u * nbufs) + 16u + 1024u;
+        total = bar_off + 8u * (3u * ns + 2u * kDkQueue + 2u * nbufs) + 16u + 4u * kDkQueue + 1024u;
     }
 };
 
@@ -288,6 +292,26 @@ __device__ __forceinline__ bool dk_wait_count(const uint32_t *p, uint32_t target
     }
     all = __shfl_sync(0xffffffffu, all ? 1 : 0, 0) != 0;
     if (all_seen && all) *all_seen = true;
+    return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+}
+
+// Lane 0 spins (bounded) until the shared word holds `item`; the result is the
+// same in every lane, and the producer's view of global memory (it saw the
+// earlier layers complete) is ordered before this warp's reads that follow.
+__device__ __forceinline__ bool dk_wait_ready(volatile int *word, int item) {
+    bool good = true;
+    if ((threadIdx.x & 31) == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (*word != item) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(&g_error_word, kErrTimeout);
+                good = false;
+                break;
+            }
+            __nanosleep(32);
+        }
+        __threadfence_block();
+    }
     return __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
 }
 
@@ -583,6 +607,8 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
     uint64_t *pfull = qempty + kDkQueue;  // consumers -> epilogue
     uint64_t *pempty = pfull + NB;
     uint32_t *conv_done = reinterpret_cast<uint32_t *>(pempty + NB);  // warps done converting
+    // per queue slot: the index of the dependent item whose inputs are final
+    volatile int *iready = reinterpret_cast<volatile int *>(conv_done + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -600,6 +626,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             mbar_init(&pempty[i], 1);
         }
         *conv_done = 0u;
+        for (int i = 0; i < kDkQueue; ++i) iready[i] = -1;
         fence_mbar_init();
     }
     __syncthreads();
@@ -648,7 +675,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         bool wrapped = false;
         int qi = 0;
         bool waited = false, ok = true, all_ready = a.total_units == 0, fenced = true;
-        uint32_t final_seen = 0;
+        uint32_t prefix_seen = 0;  // complete layers known to this producer
         const int G = (int)gridDim.x;
         int item = (int)blockIdx.x;
         DkItemRec R{};
@@ -687,6 +714,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     e.pre = pre ? 1 : 0;
                     e.chained = R.wait_tiles > 0 ? 1 : 0;
                     e.swiglu = R.wait_tiles > 0 && (R.need & 1) ? 1 : 0;
+                    e.layer = R.layer & 0xFFFF;
                 }
                 queue[q] = e;
                 mbar_arrive(&qfull[q]);
@@ -715,10 +743,11 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                                              &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
                         fenced = false;
                     }
-                } else if (R.wait_tiles > 0 && final_seen < (uint32_t)R.wait_tiles) {
-                    good = dk_wait_count(&a.ctr[kDkCtrFinal], (uint32_t)R.wait_tiles, nullptr, 0u,
+                } else if (R.wait_tiles > 0 && prefix_seen < (uint32_t)(R.layer & 0xFFFF)) {
+                    // every earlier layer complete: the prefix reaches this layer
+                    good = dk_wait_count(&a.ctr[kDkCtrPrefix], (uint32_t)(R.layer & 0xFFFF), nullptr, 0u,
                                          nullptr);
-                    if (good) final_seen = (uint32_t)R.wait_tiles;
+                    if (good) prefix_seen = (uint32_t)(R.layer & 0xFFFF);
                     fenced = false;
                 }
                 // what was observed above is read next by bulk copies (async proxy)
@@ -748,6 +777,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 // counter, which the previous grid's last CTA reset
                 next = item + G;
                 const bool in_ok = wait_inputs();
+                if (lane == 0 && in_ok && R.wait_tiles > 0) {
+                    __threadfence_block();
+                    iready[q] = item;  // the stagers may convert this item's X
+                }
                 if (lane == 0) {
                     for (int i = 0; i < pre_n; ++i) {
                         const int slot = (int)((stage + i) % NS);
@@ -769,9 +802,40 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     ok = false;
                     break;
                 }
-            } else if (!wait_inputs()) {
-                ok = false;
-                break;
+            } else {
+                if (R.wait_tiles > 0) {
+                    // a dependent item: its weights do not depend on the earlier
+                    // layers, so up to a ring's worth streams while it waits (the
+                    // slots are freed by earlier items, never by this one)
+                    const int pre_n = min(R.s1 - s, NS);
+                    for (int i = 0; i < pre_n; ++i, ++s, ++stage) {
+                        const int slot = ps;
+                        if (wrapped && !dk_warp_wait(&empty[slot], pph ^ 1u)) {
+                            ok = false;
+                            break;
+                        }
+                        if (++ps == NS) {
+                            ps = 0;
+                            pph ^= 1u;
+                            wrapped = true;
+                        }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(&wfull[slot], kDkWBytes);
+                            issue_w(slot, s);
+                        }
+                        __syncwarp();
+                    }
+                    if (!ok) break;
+                }
+                if (!wait_inputs()) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0 && R.wait_tiles > 0) {
+                    __threadfence_block();
+                    iready[q] = item;  // the stagers may convert this item's X
+                }
+                __syncwarp();
             }
             // fetched now, used after this item's stages are issued
             DkItemRec NR{};
@@ -822,6 +886,8 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         DkQEntry e;
         while (ok && dk_next_item(queue, qfull, qempty, qi, e)) {
             const int M = e.M, K = e.K;
+            const int eq = (qi - 1) % kDkQueue;  // the entry's queue slot
+            bool inputs = !e.chained;            // X of a dependent item: after iready
             for (int s = e.s0; s < e.s1; ++s) {
                 const int slot = ss;
                 const uint32_t ph = sph;
@@ -837,16 +903,19 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 // consumers to release the slot's previous round: on `empty`, not on
                 // the weights of this round -- a stager that skipped its first-round
                 // wait may reach round 1 while the slot is still in phase 0, and a
-                // parity wait on wfull would then pass a phase early.  Chained
-                // layers also wait for this round's weights, which the producer
-                // issues only once it has seen X final.
+                // parity wait on wfull would then pass a phase early.  A
+                // dependent item's X is read once the producer has seen every
+                // earlier layer complete and published the item in iready.
                 if (!fresh && !dk_warp_wait(&empty[slot], ph ^ 1u)) {
                     ok = false;
                     break;
                 }
-                if (e.chained && !dk_warp_wait(&wfull[slot], ph)) {
-                    ok = false;
-                    break;
+                if (!inputs) {
+                    if (!dk_wait_ready(&iready[eq], e.item)) {
+                        ok = false;
+                        break;
+                    }
+                    inputs = true;
                 }
                 const int valid = min(K - s * kDkStageTrits, kDkStageTrits);
                 uint8_t *dst = sslot + slot * lay.slot_b;
@@ -979,13 +1048,22 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     if (lane == 0) a.tile_ctr[e.tile_begin + e.tile] = 0u;
                 }
             }
-            if (final_tile) {
-                // the tile's outputs are stored: count it for layers that read them
-                // (by bulk copies, through the async proxy)
+            if (final_tile && a.chained) {
+                // the tile's outputs are stored: count it for its layer; the last
+                // tile of a layer advances the prefix of complete layers as far as
+                // it goes (whoever completes the next layer continues), so a
+                // dependent layer waits for every earlier layer, however the
+                // layers' tiles interleave
                 dk_fence_proxy_global();
                 __threadfence();
                 __syncwarp();
-                if (lane == 0) atomicAdd(&a.ctr[kDkCtrFinal], 1u);
+                if (lane == 0 && atomicAdd(&a.lfinal[e.layer], 1u) == a.ltiles[e.layer] - 1u) {
+                    for (int guard = 0; guard <= a.count; ++guard) {
+                        const uint32_t p = dk_ld_acquire(&a.ctr[kDkCtrPrefix]);
+                        if (p >= (uint32_t)a.count || dk_ld_acquire(&a.lfinal[p]) < a.ltiles[p]) break;
+                        atomicCAS(&a.ctr[kDkCtrPrefix], p, p + 1u);
+                    }
+                }
             }
         }
     } else {
@@ -1273,10 +1351,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         const uint32_t done = atomicAdd(&a.ctr[kDkCtrDone], 1u);
         if (done == gridDim.x - 1) {
             __threadfence();
-            a.ctr[kDkCtrFinal] = 0u;
+            a.ctr[kDkCtrPrefix] = 0u;
             a.ctr[kDkCtrItems] = 0u;
             a.ctr[kDkCtrUnitsDone] = 0u;
-            for (int l = 0; l < a.count; ++l) a.ready[l] = 0u;
+            for (int l = 0; l < a.count; ++l) a.ready[l] = a.lfinal[l] = 0u;
             a.ctr[kDkCtrDone] = 0u;
         }
     }
@@ -1342,16 +1420,13 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows) *
                  dk_stage_cost(in[l].M);
     const int cost = dk_item_cost(total);
-    bool chained = false;
-    for (int l = 0; l < count; ++l) chained = chained || in[l].reads_earlier;
     // fp16-engine items stay at 8 stages or more: their epilogue (M outputs
-    // per row) must keep up with the consumers.  In a batch with chained
-    // layers, layers run one after another, so a layer's items are sized to
-    // spread it over about one CTA per SM instead (at most 8 parts per tile
-    // for the integer engine, 2 for the fp16 engine, whose final sums of
-    // split tiles cost more).
+    // per row) must keep up with the consumers.  A layer that waits for the
+    // earlier layers starts alone, so its items are sized to spread it over
+    // about one CTA per SM instead (at most 8 parts per tile for the integer
+    // engine, 2 for the fp16 engine, whose final sums of split tiles cost more).
     auto target_of = [&](const DkHostLayer &h) {
-        if (chained) {
+        if (h.reads_earlier) {
             const int64_t units = (int64_t)stages_of(h) * ((h.N + kDkRows - 1) / kDkRows);
             const int t = (int)((units + kDkRefSms - 1) / kDkRefSms);
             const int min_t = (stages_of(h) + (h.M > kDkImmaMaxM ? 1 : 7)) / (h.M > kDkImmaMaxM ? 2 : 8);
@@ -1426,7 +1501,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
                 r.ldy = (int)h.ldy;
                 r.parts = parts;
                 r.tile_begin = tile_begin;
-                r.wait_tiles = h.reads_earlier ? tile_begin : 0;
+                r.wait_tiles = h.reads_earlier ? 1 : 0;
                 r.need = h.reads_earlier ? (h.swiglu ? 1 : 0) : stages * h.M;
                 r.bstride = bstride;
                 items->push_back(r);
@@ -1490,6 +1565,8 @@ inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int
     a.items = reinterpret_cast<const DkItemRec *>(b + wl.items);
     a.units = reinterpret_cast<const DkUnitRec *>(b + wl.units);
     a.ready = reinterpret_cast<uint32_t *>(b + wl.ready);
+    a.lfinal = a.ready + count;
+    a.ltiles = a.ready + 2 * count;
     a.tile_ctr = reinterpret_cast<uint32_t *>(b + wl.tiles);
     a.partials = reinterpret_cast<int64_t *>(b + wl.partials);
     a.count = count;

@@ -160,7 +160,13 @@ int plan_decode2(int count, const std::vector<tlk::GpHostLayer> &h, void *dWorks
     if (e == cudaSuccess && !units.empty())
         e = cudaMemcpy(ws + wl.units, units.data(), sizeof(tlk::DkUnitRec) * units.size(),
                        cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemset(ws + wl.ready, 0, wl.partials - wl.ready);  // ready, tiles
+    // ready, per-layer final tiles, per-layer tile counts, tile counters
+    if (e == cudaSuccess) e = cudaMemset(ws + wl.ready, 0, wl.partials - wl.ready);
+    std::vector<uint32_t> ltiles(count);
+    for (int l = 0; l < count; ++l) ltiles[l] = (uint32_t)((dh[l].N + tlk::kDkRows - 1) / tlk::kDkRows);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(ws + wl.ready + 8 * (size_t)count, ltiles.data(), 4 * (size_t)count,
+                       cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e);
     plan->fmt = TL_FMT_2BIT;

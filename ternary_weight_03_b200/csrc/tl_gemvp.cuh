@@ -700,6 +700,7 @@ struct GpSchedule {
 inline GpSchedule gp_schedule(int fmt, int count, const GpHostLayer *in, GpLayer *out) {
     GpSchedule sc;
     sc.count = count;
+    bool after_dependent = false;
     for (int l = 0; l < count; ++l) {
         const GpHostLayer &h = in[l];
         GpLayer &L = out[l];
@@ -720,7 +721,11 @@ inline GpSchedule gp_schedule(int fmt, int count, const GpHostLayer *in, GpLayer
         L.tiles = (h.N + kGpRows - 1) / kGpRows;
         L.item_begin = sc.total_items;
         L.tile_begin = sc.total_tiles;
-        L.wait_tiles = h.reads_earlier ? sc.total_tiles : 0;
+        // A layer after a dependent one waits too: the final-tile counter only
+        // says how many tiles are final, so a later independent layer's tiles
+        // must not be able to stand in for an earlier layer's missing ones.
+        after_dependent = after_dependent || h.reads_earlier;
+        L.wait_tiles = after_dependent ? sc.total_tiles : 0;
         L.part_off = sc.floats;
         if (L.parts > 1) sc.floats += (int64_t)L.tiles * L.parts * kGpRows * h.M;
         sc.total_items += L.tiles * L.parts;

@@ -134,10 +134,11 @@ def _ws2_expected(layers):
     counters, one 128-byte tensor map per layer, a 96-byte record per work item
     (256-row tile x K-part of 2..16 stages of 512 trits), a 48-byte record per
     conversion unit (stage x token of a layer that reads no earlier output), a
-    u32 per layer and per tile, 8-byte partials of split tiles, and the
+    u32 per tile, three u32 per layer (ready units, final tiles, tiles), 8-byte
+    partials of split tiles, and the
     converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage).
-    With a chained layer in the batch, a layer's items are sized to spread it
-    over about 148 CTAs (at most 8 parts per tile, 2 for M > 2).  Independent
+    A layer with a dependency has its items sized to spread it over about
+    148 CTAs (at most 8 parts per tile, 2 for M > 2).  Independent
     layers with the same X (pointer, ldx, K, M) share the first one's
     conversion (no units or converted activations of their own)."""
     items = units = tiles = slots = staged = 0
@@ -145,11 +146,10 @@ def _ws2_expected(layers):
     cm = lambda d: 1 if d["M"] <= 2 else 2  # relative cost of a stage
     total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
     cost = min(16, max(4, total // (4 * 148)))  # cost per item
-    chained = any(d.get("flags", 0) for d in layers)
     seen = set()
     for d in layers:
         stages = stg(d)
-        if chained:
+        if d.get("flags", 0):
             target = -(-stages * -(-d["N"] // 256) // 148)
             min_t = -(-stages // (2 if d["M"] > 2 else 8))
             target = max(target, min_t, 1)
@@ -170,7 +170,7 @@ def _ws2_expected(layers):
         if parts > 1:
             slots += t * parts * 256 * d["M"]
     off = 256
-    for size in (128 * len(layers), 96 * items, 48 * units, 4 * len(layers), 4 * tiles, 8 * slots,
+    for size in (128 * len(layers), 96 * items, 48 * units, 12 * len(layers), 4 * tiles, 8 * slots,
                  staged):
         off = _up(off + size)
     return off

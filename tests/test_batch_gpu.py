@@ -405,3 +405,54 @@ def test_layers_sharing_x(M):
     assert tl.device_status() == 0
     for T, X, a, dY, N in cases:
         _check_layer(T, X, a, dY, N, M)
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+def test_dependent_layer_before_independent_ones(fmt):
+    """A slow producer (one tile, long K), a layer reading its output, then
+    sixteen small independent layers that finish quickly.  The dependent
+    layer must see its producer complete however the layers' tiles
+    interleave (a count of final tiles alone would let the small layers'
+    tiles stand in for the producer's).  Repeated runs agree bit for bit."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    M, K0, N0 = 2, 20000, 256
+    T0 = synth.trits(120, N0, K0)
+    X0 = synth.activations(121, M, K0)
+    T1 = synth.trits(122, 300, N0)
+    a0, a1 = 0.004, 0.03
+    dX0 = torch.from_numpy(X0).cuda()
+    Y0 = torch.full((M, N0), float("nan"), dtype=torch.float16, device="cuda")
+    Y1 = torch.full((M, 304), float("nan"), dtype=torch.float16, device="cuda")
+    pk = lambda T: torch.from_numpy(tl.pack(fmt, T)).cuda()
+    specs = [(pk(T0), a0, dX0, K0, Y0), (pk(T1), a1, Y0, N0, Y1, tl.LAYER_READS_EARLIER)]
+    small = []
+    for i in range(16):
+        T = synth.trits(130 + i, 64, 128)
+        X = synth.activations(150 + i, M, 128)
+        Y = torch.full((M, 64), float("nan"), dtype=torch.float16, device="cuda")
+        specs.append((pk(T), 0.05, torch.from_numpy(X).cuda(), 128, Y))
+        small.append((T, X, Y))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    outs = []
+    for _ in range(3):
+        Y0.fill_(float("nan"))
+        Y1.fill_(float("nan"))
+        tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+        assert tl.device_status() == 0
+        outs.append(Y1.cpu().numpy().view(np.uint16).copy())
+    for o_ in outs[1:]:
+        assert np.array_equal(o_, outs[0])
+    o = oracle.get()
+    ref0 = o.linear(T0, X0, a0, nthreads=8)
+    y0 = Y0.cpu().numpy()
+    assert (np.abs(y0.astype(np.float64) - ref0) <= oracle.tolerance(ref0, X0, a0)).all()
+    ref1 = o.linear(T1, y0, a1, nthreads=8)
+    ulp = np.spacing(np.abs(y0)).astype(np.float64)
+    tol = oracle.tolerance(ref1, y0, a1) + abs(a1) * ulp.sum(axis=1)[:, None]
+    got = Y1[:, :300].float().cpu().numpy().astype(np.float64)
+    assert (np.abs(got - ref1) <= tol).all()
+    for T, X, Y in small:
+        ref = o.linear(T, X, 0.05)
+        assert (np.abs(Y.float().cpu().numpy() - ref) <= oracle.tolerance(ref, X, 0.05)).all()
