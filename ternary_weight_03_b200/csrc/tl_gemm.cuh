@@ -385,13 +385,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
                                            __uint_as_float(v[4 * c4 + 2]),
                                            __uint_as_float(v[4 * c4 + 3]));
             }
-            // reduce the units this CTA owns, in rank order
+            // reduce the units this CTA owns, in rank order; the owned units of
+            // a quarter (c = first, first + S, ...) go to its warps in turn
             if (mbar_wait_cluster(redbar, 0)) {
                 const int n = n0 + quarter * 32 + lane;
+                const int first = (int)((rank + S - (uint32_t)(quarter * kChunks) % S) % S);
+                int turn = 0;
 #pragma unroll 1
-                for (int c = half; c < kChunks; c += kGemmDecSets) {
-                    const int u = quarter * kChunks + c;
-                    if ((uint32_t)u % S != rank) continue;
+                for (int c = first; c < kChunks; c += (int)S, ++turn) {
+                    if (turn % kGemmDecSets != half) continue;
+                    const int u = quarter * kChunks + c;  // u mod S == rank
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tmem + lane_addr + c * 32, v);
                     tc_wait_ld();
