@@ -28,8 +28,8 @@
 // shares one output tile, rank r taking K-steps [r nk / S, (r + 1) nk / S)
 // (1.6-bit: whole 320-trit blocks, so every rank starts on a block).
 // After one cluster barrier (every ring is then idle), the accumulator is
-// cut into units of 32 rows (a TMEM lane quarter) x 32 columns; unit u is
-// owned by rank u mod S.  Each CTA pushes the units it does not own from
+// cut into units of 32 rows (a TMEM lane quarter) x 16 columns; unit u is
+// owned by rank u mod S, and a quarter's owned units go to its warps in turn.  Each CTA pushes the units it does not own from
 // TMEM into the owner's activation ring with st.async, and the owner sums
 // the S partials of its units in rank order -- deterministic, no global
 // workspace.
@@ -182,9 +182,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
     const int kb = KU * (int)(((int64_t)nu * rank) / S);
     const int ke = min(nk_all, KU * (int)(((int64_t)nu * (rank + 1)) / S));
     const int nk = ke - kb;
-    // accumulator units: 4 lane quarters x kChunks column chunks of kChunkW
-    constexpr int kChunkW = BN < 32 ? BN : 32;
-    constexpr int kChunks = (BN + 31) / 32;
+    // split-K accumulator units: 4 lane quarters x kChunks column chunks of kChunkW
+    constexpr int kChunkW = 16;
+    constexpr int kChunks = BN / kChunkW;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
@@ -371,8 +371,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
                 const int u = quarter * kChunks + c;
                 const uint32_t owner = (uint32_t)u % S;
                 if (owner == rank) continue;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + lane_addr + c * 32, v);
+                uint32_t v[kChunkW];
+                tmem_ld_32x32b_x16(tmem + lane_addr + c * kChunkW, v);
                 tc_wait_ld();
                 const uint32_t slot = rank * per + (uint32_t)u / S;
                 const uint32_t dst = mapa_shared(
@@ -395,8 +395,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
                 for (int c = first; c < kChunks; c += (int)S, ++turn) {
                     if (turn % kGemmDecSets != half) continue;
                     const int u = quarter * kChunks + c;  // u mod S == rank
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem + lane_addr + c * 32, v);
+                    uint32_t v[kChunkW];
+                    tmem_ld_32x32b_x16(tmem + lane_addr + c * kChunkW, v);
                     tc_wait_ld();
 #pragma unroll
                     for (int c4 = 0; c4 < kChunkW / 4; ++c4) {
@@ -421,7 +421,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ 
                         if (n < N) {
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
-                                const int m = m0 + c * 32 + 4 * c4 + j;
+                                const int m = m0 + c * kChunkW + 4 * c4 + j;
                                 if (m < M)
                                     Y[(int64_t)m * ldy + n] = f32_to_f16_bits(alpha * a[j]);
                             }
@@ -491,12 +491,12 @@ inline int gemm_resident(int dev, int S, size_t smem) {
 
 // Split-K factor: the largest S in {1, 2, 4, 8} such that the S-CTA clusters
 // of all output tiles are resident at once, S divides the accumulator's
-// 4 x ceil(BN / 32) units and every rank keeps at least one K-range unit
+// 4 x BN / 16 units and every rank keeps at least one K-range unit
 // (a K-step of 64 trits; 1.6-bit: a packed block of 320 trits).
 template <int FMT, int BN>
 inline int gemm_split(int dev, int M, int N, int K, size_t smem) {
     const int64_t tiles = (int64_t)((N + kGemmRows - 1) / kGemmRows) * ((M + BN - 1) / BN);
-    const int units = 4 * ((BN + 31) / 32);
+    const int units = 4 * (BN / 16);
     const int ku = GemmSmem<FMT>::ksteps_per_w * kGemmKStep;
     const int nk = (K + ku - 1) / ku;
     int S = 1;
