@@ -1529,13 +1529,41 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     // launch's tail) are the cheapest.  A part of a split tile also counts
     // the finish its tile may need (one round of loads per token and per
     // four parts, about a stage each), so split tiles finish early.
-    if (!sc.chained)
+    if (!sc.chained) {
         std::stable_sort(items->begin(), items->end(), [](const DkItemRec &x, const DkItemRec &y) {
             auto cost = [](const DkItemRec &r) {
                 return (r.s1 - r.s0) * dk_stage_cost(r.M) + (r.parts > 1 ? r.M * ((r.parts + 3) / 4) : 0);
             };
             return cost(x) > cost(y);
         });
+        return sc;
+    }
+    // With dependencies, a dependent layer's items must follow every item of
+    // the earlier layers (then everything it waits for was handed out before
+    // it).  Within that rule, each dependent layer's items are handed out
+    // after the independent layers that follow it, just before the next
+    // dependent layer's: a CTA that takes a dependent item then mostly finds
+    // its inputs complete instead of waiting while independent work remains.
+    // A chain of dependent layers keeps its order.
+    std::vector<DkItemRec> ordered;
+    ordered.reserve(items->size());
+    size_t i = 0, pending_begin = 0, pending_end = 0;  // the held-back dependent layer
+    while (i < items->size()) {
+        const int layer = (*items)[i].layer & 0xFFFF;
+        size_t j = i;
+        while (j < items->size() && ((*items)[j].layer & 0xFFFF) == layer) ++j;
+        if ((*items)[i].wait_tiles > 0) {
+            ordered.insert(ordered.end(), items->begin() + pending_begin,
+                           items->begin() + pending_end);
+            pending_begin = i;
+            pending_end = j;
+        } else {
+            ordered.insert(ordered.end(), items->begin() + i, items->begin() + j);
+        }
+        i = j;
+    }
+    ordered.insert(ordered.end(), items->begin() + pending_begin, items->begin() + pending_end);
+    items->swap(ordered);
     return sc;
 }
 
