@@ -391,8 +391,8 @@ __device__ __forceinline__ void dk_read_word_glu(const uint16_t *src, const uint
     for (int i = 0; i < 8; ++i) {
         const float2 gf = __half22float2(*reinterpret_cast<const __half2 *>(&g[i]));
         const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&u[i]));
-        const float a = gf.x / (1.0f + expf(-gf.x)) * uf.x;
-        const float b = gf.y / (1.0f + expf(-gf.y)) * uf.y;
+        const float a = __fdividef(gf.x, 1.0f + __expf(-gf.x)) * uf.x;
+        const float b = __fdividef(gf.y, 1.0f + __expf(-gf.y)) * uf.y;
         const __half2 h = __floats2half2_rn(a, b);
         r[i] = *reinterpret_cast<const uint32_t *>(&h);
     }
