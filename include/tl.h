@@ -164,21 +164,20 @@ typedef struct tl_gemv_plan {
     uint64_t generation; /* 0, or the static plan's number (tl_gemv_batch_plan_static) */
 } tl_gemv_plan;
 
-/* Workspace bytes a batch needs.  2-bit: counters, one TMA descriptor per
- * layer, a 96-byte record per work item (256 output rows x 4096..8192 trits
- * of K), the layers' activations converted once into the tensor-core operand
- * layout (per 512 trits of K: 4 KB at M = 1, 8 KB at M = 2, 1 KB per token
- * rounded up to even at M >= 3, plus 64 B; none for TL_LAYER_READS_EARLIER
- * layers, which convert on chip) with a 48-byte record per 512 trits and
- * token, and 8-byte partial sums of rows split into K-parts (N * M * 8 bytes
- * per part).  1.6-bit: the layer table and one TMA descriptor per layer
- * (~200 B per layer), counters, and fp32 partial sums of the layers whose
- * rows are split across CTAs (about N * M * 4 * K / 2048 bytes per such
- * layer).  Validates the batch like tl_gemv_batch_plan.  Pure host
+/* Workspace bytes a batch needs: counters, one TMA descriptor per layer, a
+ * 96-byte record per work item (256 output rows x a K-part of whole stages;
+ * a stage is 128 packed bytes per row, 512 trits at 2 bits or 640 at 1.6
+ * bits), the layers' activations converted once into the tensor-core
+ * operand layout (per stage 64 B plus 8 B per trit x M at M <= 2, 2 B per
+ * trit x M rounded up to even at M >= 3; none for TL_LAYER_READS_EARLIER
+ * layers, which convert on chip) with a 48-byte record per stage and token,
+ * and 8-byte partial sums of rows split into K-parts (N * M * 8 bytes per
+ * part).  Validates the batch like tl_gemv_batch_plan.  Pure host
  * function. */
 int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes);
 
-/* Plans count (1 .. TL_GEMV_BATCH_MAX) decode-shaped layers of one format
+/* Plans count (1 .. TL_GEMV_BATCH_MAX) decode-shaped layers of one format (2-
+ * or 1.6-bit, both run by the same persistent kernel)
  * for single-launch execution by tl_gemv_batch_run.  Every layer follows the
  * argument rules of tl_gemv; layers[] is host memory, read before the call
  * returns.  Writes the layer table and the layers' TMA descriptors into
@@ -192,7 +191,7 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
  * Y, so it may consume their outputs (a chain of layers); without the flag,
  * X must not be written by any layer of the batch.  No Y may overlap another
  * layer's Y, X or T.
- * SwiGLU input (2-bit only; TL_LAYER_SWIGLU_INPUT together with
+ * SwiGLU input (TL_LAYER_SWIGLU_INPUT together with
  * TL_LAYER_READS_EARLIER): row m of dX holds a gated unit's two inputs, the
  * gate values g in elements [0, K) and the up values u in [K, 2K) (typically
  * the outputs of two earlier layers writing the halves of one buffer), and
@@ -200,13 +199,13 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
  * exp(-g)), evaluated in fp32 -- the gated feed-forward unit of a LLaMA-style
  * decoder fused into its down projection, so the product never goes to
  * memory.  Needs ldx >= 2 K and K % 8 == 0 (else TL_ERR_INVALID_ARG /
- * TL_ERR_ALIGN); the 1.6-bit batch returns TL_ERR_UNSUPPORTED.
+ * TL_ERR_ALIGN).
  * Independent layers with the same X (pointer, ldx, K and M; no
  * TL_LAYER_READS_EARLIER), such as the Q, K and V projections of one token
  * batch, share one conversion of X: it is staged once per launch, and each
  * layer keeps its own alpha.
  * Errors: TL_ERR_INVALID_ARG (bad layer, count or workspace too small),
- * TL_ERR_ALIGN, TL_ERR_UNSUPPORTED, TL_ERR_CUDA. */
+ * TL_ERR_ALIGN, TL_ERR_CUDA. */
 int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dWorkspace,
                        size_t workspace_bytes, tl_gemv_plan *plan);
 

@@ -72,8 +72,7 @@ namespace tlk {
 constexpr int kDkTiles = 16;                             // 16-row MMA tiles per item
 constexpr int kDkRows = 16 * kDkTiles;                   // 256 weight rows per item
 constexpr int kDkStageW = 128;                           // packed bytes per row per stage (one box)
-constexpr int kDkStageTrits = 4 * kDkStageW;             // 512 activations per stage
-constexpr int kDkWords = kDkStageW / 4;                  // 32 words of 16 trits per row per stage
+constexpr int kDkWords = kDkStageW / 4;                  // 32 packed words per row per stage
 constexpr int kDkWBytes = kDkRows * kDkStageW;           // 32 KB of weights per stage
 constexpr int kDkConsumers = 16;
 constexpr int kDkStagers = 3;
@@ -97,11 +96,20 @@ constexpr int kDkCtrDone = 2;       // CTAs that have finished
 constexpr int kDkCtrItems = 3;      // items handed out beyond the first 2 gridDim.x
 constexpr int kDkCtrUnitsDone = 5;  // CTAs whose conversion units are all written
 
+// Activations per stage: 128 packed bytes of 4 (2-bit) or 5 (1.6-bit) trits.
+__host__ __device__ constexpr int dk_trits(int fmt) { return fmt == 2 ? 4 * kDkStageW : 5 * kDkStageW; }
 // Bytes of converted B operands of one stage of a layer with M tokens: the
-// integer engine needs 4 KB per column group (2 groups at M = 2), the fp16
-// engine 1 KB per token (tokens rounded up to even).
-__host__ __device__ constexpr uint32_t dk_stage_b(int M) {
-    return M <= 1 ? 4096u : (M == 2 ? 8192u : 1024u * (uint32_t)(M + (M & 1)));
+// integer engine needs one byte per activation and column of a group of 8
+// (2 groups at M = 2), the fp16 engine 2 bytes per activation and token
+// (tokens rounded up to even).
+__host__ __device__ constexpr uint32_t dk_stage_b(int fmt, int M) {
+    return M <= 2 ? 8u * (uint32_t)dk_trits(fmt) * (uint32_t)M
+                  : 2u * (uint32_t)dk_trits(fmt) * (uint32_t)(M + (M & 1));
+}
+// The largest stage of a batch whose layers have at most maxM tokens.
+__host__ __device__ constexpr uint32_t dk_slot_b(int fmt, int maxM) {
+    return dk_stage_b(fmt, maxM < 2 ? maxM : 2) > dk_stage_b(fmt, maxM) ? dk_stage_b(fmt, maxM < 2 ? maxM : 2)
+                                                                      : dk_stage_b(fmt, maxM);
 }
 // Consumer -> epilogue buffer: [token][warp][tile][row] of int64 (M <= 2) or fp32.
 __host__ __device__ constexpr uint32_t dk_part_bytes(int maxM) {
@@ -198,8 +206,8 @@ struct DkQEntry {
 
 struct DkLayout {
     uint32_t ns, nbufs, slot_b, parts, w_off, st_off, part_off, q_off, bar_off, total;
-    __host__ __device__ explicit DkLayout(int maxM) {
-        slot_b = (maxM <= 1 ? 4096u : 8192u) + kDkMetaBytes;  // [meta][B]
+    __host__ __device__ DkLayout(int fmt, int maxM) {
+        slot_b = dk_slot_b(fmt, maxM) + kDkMetaBytes;  // [meta][B]
         parts = dk_part_bytes(maxM);
         nbufs = parts <= 8192u ? (uint32_t)kDkMaxPartBufs : 2u;
         const uint32_t per_stage = (uint32_t)kDkWBytes + slot_b;
@@ -382,20 +390,21 @@ __device__ __forceinline__ void dk_read_word(const uint16_t *src, int w, int val
 // The same for a SwiGLU input: element e of the word is
 // fp16_rn(silu(g_e) * u_e) in fp32, g from src and u from up = src + K (the
 // row's second half); zero at e >= valid.
+__device__ __forceinline__ uint32_t dk_glu2(uint32_t g, uint32_t u) {
+    const float2 gf = __half22float2(*reinterpret_cast<const __half2 *>(&g));
+    const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&u));
+    const float a = __fdividef(gf.x, 1.0f + __expf(-gf.x)) * uf.x;
+    const float b = __fdividef(gf.y, 1.0f + __expf(-gf.y)) * uf.y;
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
 __device__ __forceinline__ void dk_read_word_glu(const uint16_t *src, const uint16_t *up, int w,
                                                  int valid, uint32_t (&r)[8]) {
     uint32_t g[8], u[8];
     dk_read_word(src, w, valid, g);
     dk_read_word(up, w, valid, u);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float2 gf = __half22float2(*reinterpret_cast<const __half2 *>(&g[i]));
-        const float2 uf = __half22float2(*reinterpret_cast<const __half2 *>(&u[i]));
-        const float a = __fdividef(gf.x, 1.0f + __expf(-gf.x)) * uf.x;
-        const float b = __fdividef(gf.y, 1.0f + __expf(-gf.y)) * uf.y;
-        const __half2 h = __floats2half2_rn(a, b);
-        r[i] = *reinterpret_cast<const uint32_t *>(&h);
-    }
+    for (int i = 0; i < 8; ++i) r[i] = dk_glu2(g[i], u[i]);
 }
 // One word of a stage's activations: plain, or the SwiGLU product (up != null).
 __device__ __forceinline__ void dk_load_word(const uint16_t *src, const uint16_t *up, int w,
@@ -487,6 +496,155 @@ __device__ __forceinline__ void dk_conv_hmma(const uint16_t *src, const uint16_t
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
     if (lane == 0) reinterpret_cast<float *>(meta)[m] = sx;
+}
+
+// ---- base 3 (1.6-bit) ----
+// A packed byte v = sum_i d_i 3^i (d = t + 1) holds five trits; with
+// q_i = floor(v / 3^i) (q_0 = v), d_i = q_i - 3 q_{i+1} and d_4 = q_4, so for
+// the activations xi_{5b+i} of byte b
+//   sum_i d_i xi_{5b+i} = q_0 xi_{5b} + sum_{p=1..4} q_p (xi_{5b+p} - 3 xi_{5b+p-1}).
+// The quotients of the four bytes of a word come out of 16-bit lanes: for
+// v < 256, floor(85 (v + 1) / 256) = floor(v / 3) (exact for v < 243, the
+// valid codes), and 85 (v + 1) < 2^16, so one IMAD serves two bytes and the
+// quotient is the product's high byte.
+
+// The 20 activations of packed word w of a base-3 stage (elements 20w ..
+// 20w + 19 of a stage that starts at src), zero at elements >= valid.  Only
+// whole 4-element groups that start below `valid` are read (ldx is a multiple
+// of 8 and >= K, so they stay inside the row).
+__device__ __forceinline__ void dk_read20(const uint16_t *src, int w, int valid, uint32_t (&r)[10]) {
+#pragma unroll
+    for (int i = 0; i < 5; ++i) {
+        const int e = 20 * w + 4 * i;
+        uint2 v = make_uint2(0u, 0u);
+        if (e < valid) v = *reinterpret_cast<const uint2 *>(src + e);
+        const int keep = valid - e;
+        if (keep < 4) {
+            v.x &= (keep > 0 ? 0x0000FFFFu : 0u) | (keep > 1 ? 0xFFFF0000u : 0u);
+            v.y &= (keep > 2 ? 0x0000FFFFu : 0u);
+        }
+        r[2 * i] = v.x;
+        r[2 * i + 1] = v.y;
+    }
+}
+// The same, plain or as the SwiGLU product (up != null).
+__device__ __forceinline__ void dk_load20(const uint16_t *src, const uint16_t *up, int w, int valid,
+                                          uint32_t (&r)[10]) {
+    dk_read20(src, w, valid, r);
+    if (up) {
+        uint32_t u[10];
+        dk_read20(up, w, valid, u);
+#pragma unroll
+        for (int i = 0; i < 10; ++i) r[i] = dk_glu2(r[i], u[i]);
+    }
+}
+// Element e (0..19) of a word read by dk_read20 as the halves of r.
+template <int E0, int E1>
+__device__ __forceinline__ uint32_t dk_pair20(const uint32_t (&r)[10]) {
+    return prmt(r[E0 >> 1], r[E1 >> 1], ((E0 & 1) ? 0x32u : 0x10u) | ((E1 & 1) ? 0x7600u : 0x5400u));
+}
+
+// Integer engine, base 3: offset of the 8-byte B entry of (half v, word pair
+// pr, position p, column col, lane column c): words 2pr and 2pr + 1 of chunk
+// 4v + c, four bytes each.  A quarter-warp reads 64 contiguous bytes.
+__host__ __device__ constexpr uint32_t dk_i3off(int v, int pr, int p, int col, int c) {
+    return (uint32_t)((col >> 3) * 5 * 1024 + ((((v * 2 + pr) * 5 + p) * 8 + (col & 7)) * 4 + c) * 8);
+}
+// fp16 engine, base 3: offset of the 8-byte B entry of (half v, word i of the
+// chunk, digit p, token m, lane column c), Mp tokens rounded up to even.
+__host__ __device__ constexpr uint32_t dk_h3off(int v, int i, int p, int m, int c, int Mp) {
+    return (uint32_t)(((((v * 4 + i) * 5 + p) * Mp + m) * 4 + c) * 8);
+}
+
+// One warp converts one base-3 stage of token m for the integer engine.  Lane
+// w takes packed word w (bytes 4w .. 4w + 3).  With xi = x 2^24 (an integer,
+// |xi| < 2^40), position p of byte b has the B operand
+//   p = 0: xi_{5b} + 2^42,   p >= 1: xi_{5b+p} - 3 xi_{5b+p-1} + 2^42,
+// a natural number below 2^43 stored as six u8 planes; the 2^42 offsets come
+// back out as 2^42 times the ones column's sum of A.  Q = sum xi into meta[m]
+// (exact in a double: below 2^50).
+__device__ __forceinline__ void dk_conv_imma3(const uint16_t *src, const uint16_t *up, int valid,
+                                              int m, int M, uint8_t *dstB, uint8_t *meta, int lane) {
+    const int w = lane, ch = w >> 2, i = w & 3, v = ch >> 2, c = ch & 3, pr = i >> 1, hf = i & 1;
+    uint32_t r[10];
+    dk_load20(src, up, w, valid, r);
+    int64_t xi[20];
+    double qd = 0.0;
+#pragma unroll
+    for (int k = 0; k < 10; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[k]));
+        xi[2 * k] = (int64_t)(f.x * 16777216.0f);  // exact: a binary16 times 2^24
+        xi[2 * k + 1] = (int64_t)(f.y * 16777216.0f);
+        qd += (double)xi[2 * k] + (double)xi[2 * k + 1];
+    }
+    const int ones = dk_ones_col(M);
+#pragma unroll
+    for (int p = 0; p < 5; ++p) {
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t b = (p == 0 ? xi[5 * e] : xi[5 * e + p] - 3 * xi[5 * e + p - 1]) + (1ll << 42);
+            lo[e] = (uint32_t)b;
+            hi[e] = (uint32_t)(b >> 32);
+        }
+        // plane j's word holds byte j of the four bytes' operands
+        const uint32_t a01 = prmt(lo[0], lo[1], 0x5140u), a23 = prmt(lo[2], lo[3], 0x5140u);
+        const uint32_t c01 = prmt(lo[0], lo[1], 0x7362u), c23 = prmt(lo[2], lo[3], 0x7362u);
+        const uint32_t h01 = prmt(hi[0], hi[1], 0x5140u), h23 = prmt(hi[2], hi[3], 0x5140u);
+        const uint32_t pl[6] = {prmt(a01, a23, 0x5410u), prmt(a01, a23, 0x7632u),
+                                prmt(c01, c23, 0x5410u), prmt(c01, c23, 0x7632u),
+                                prmt(h01, h23, 0x5410u), prmt(h01, h23, 0x7632u)};
+#pragma unroll
+        for (int j = 0; j < 6; ++j)
+            *reinterpret_cast<uint32_t *>(dstB + dk_i3off(v, pr, p, dk_col(m, j), c) + 4 * hf) = pl[j];
+        if (m == 0)
+            *reinterpret_cast<uint32_t *>(dstB + dk_i3off(v, pr, p, ones, c) + 4 * hf) = 0x01010101u;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) qd += __shfl_xor_sync(0xffffffffu, qd, o);
+    if (lane == 0) reinterpret_cast<int64_t *>(meta)[m] = (int64_t)qd;
+}
+
+// One warp converts one base-3 stage of token m for the fp16 engine: per word
+// and digit p the pairs (x_p, x_{10+p}) and (x_{5+p}, x_{15+p}) of the word's
+// elements (bytes 0 and 2, bytes 1 and 3), and sum x into meta[m] (fp32).
+__device__ __forceinline__ void dk_conv_hmma3(const uint16_t *src, const uint16_t *up, int valid,
+                                              int m, int Mp, uint8_t *dstB, uint8_t *meta, int lane) {
+    const int w = lane, ch = w >> 2, i = w & 3, v = ch >> 2, c = ch & 3;
+    uint32_t r[10];
+    dk_load20(src, up, w, valid, r);
+    float sx = 0.f;
+#pragma unroll
+    for (int k = 0; k < 10; ++k) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r[k]));
+        sx += f.x + f.y;
+    }
+    uint2 *d = reinterpret_cast<uint2 *>(dstB);
+    d[dk_h3off(v, i, 0, m, c, Mp) / 8] = make_uint2(dk_pair20<0, 10>(r), dk_pair20<5, 15>(r));
+    d[dk_h3off(v, i, 1, m, c, Mp) / 8] = make_uint2(dk_pair20<1, 11>(r), dk_pair20<6, 16>(r));
+    d[dk_h3off(v, i, 2, m, c, Mp) / 8] = make_uint2(dk_pair20<2, 12>(r), dk_pair20<7, 17>(r));
+    d[dk_h3off(v, i, 3, m, c, Mp) / 8] = make_uint2(dk_pair20<3, 13>(r), dk_pair20<8, 18>(r));
+    d[dk_h3off(v, i, 4, m, c, Mp) / 8] = make_uint2(dk_pair20<4, 14>(r), dk_pair20<9, 19>(r));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sx += __shfl_xor_sync(0xffffffffu, sx, o);
+    if (lane == 0) reinterpret_cast<float *>(meta)[m] = sx;
+}
+
+// One stage of token m in the B layout of the item's engine.
+template <int FMT>
+__device__ __forceinline__ void dk_convert(const uint16_t *src, const uint16_t *up, int valid, int m,
+                                           int M, uint8_t *slot, int lane) {
+    if constexpr (FMT == 2) {
+        if (M <= kDkImmaMaxM)
+            dk_conv_imma(src, up, valid, m, M, slot + kDkMetaBytes, slot, lane);
+        else
+            dk_conv_hmma(src, up, valid, m, M + (M & 1), slot + kDkMetaBytes, slot, lane);
+    } else {
+        if (M <= kDkImmaMaxM)
+            dk_conv_imma3(src, up, valid, m, M, slot + kDkMetaBytes, slot, lane);
+        else
+            dk_conv_hmma3(src, up, valid, m, M + (M & 1), slot + kDkMetaBytes, slot, lane);
+    }
 }
 
 // The last part of a split tile adds the tile's parts in part order and stores
@@ -587,10 +745,11 @@ __device__ __noinline__ void dk_finalize(const int64_t *base, int cnt, int parts
 
 // kGlu: the batch has SwiGLU-input layers (a separate instantiation, so that
 // the conversion's fp32 silu code is not part of every other batch's kernel).
-template <bool kGlu>
+template <int FMT, bool kGlu>
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
+    constexpr int TS = dk_trits(FMT);  // activations per stage
     extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
-    const DkLayout lay(a.maxM);
+    const DkLayout lay(FMT, a.maxM);
     const int NS = (int)lay.ns;
     // 1024-byte alignment for the 128-byte swizzle of the weight boxes
     uint8_t *smem = dk_smem_raw + ((1024u - (smem_u32(dk_smem_raw) & 1023u)) & 1023u);
@@ -643,13 +802,9 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         for (int u = crank * (int)gridDim.x + (int)blockIdx.x; u < a.total_units;
              u += (int)gridDim.x * kConv) {
             const DkUnitRec U = dk_load_rec<DkUnitRec, 3>(a.units, u);
-            const int valid = min(U.K - U.stage * kDkStageTrits, kDkStageTrits);
-            const uint16_t *src = U.X + (int64_t)U.m * U.ldx + (int64_t)U.stage * kDkStageTrits;
-            if (U.M <= kDkImmaMaxM)
-                dk_conv_imma(src, nullptr, valid, U.m, U.M, U.dst + kDkMetaBytes, U.dst, lane);
-            else
-                dk_conv_hmma(src, nullptr, valid, U.m, U.M + (U.M & 1), U.dst + kDkMetaBytes, U.dst,
-                             lane);
+            const int valid = min(U.K - U.stage * TS, TS);
+            const uint16_t *src = U.X + (int64_t)U.m * U.ldx + (int64_t)U.stage * TS;
+            dk_convert<FMT>(src, nullptr, valid, U.m, U.M, U.dst, lane);
             // the converted unit is read by bulk copies of other CTAs
             dk_fence_proxy_global();
             __threadfence();
@@ -917,15 +1072,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                     inputs = true;
                 }
-                const int valid = min(K - s * kDkStageTrits, kDkStageTrits);
+                const int valid = min(K - s * TS, TS);
                 uint8_t *dst = sslot + slot * lay.slot_b;
                 for (int m = 0; m < M; ++m) {
-                    const uint16_t *src = e.X + (int64_t)m * e.ldx + (int64_t)s * kDkStageTrits;
+                    const uint16_t *src = e.X + (int64_t)m * e.ldx + (int64_t)s * TS;
                     const uint16_t *up = kGlu && e.swiglu ? src + K : nullptr;  // [gate | up] rows
-                    if (M <= kDkImmaMaxM)
-                        dk_conv_imma(src, up, valid, m, M, dst + kDkMetaBytes, dst, lane);
-                    else
-                        dk_conv_hmma(src, up, valid, m, M + (M & 1), dst + kDkMetaBytes, dst, lane);
+                    dk_convert<FMT>(src, up, valid, m, M, dst, lane);
                 }
 #ifdef TL_DEBUG_HOOKS
                 // the hook: CTA 0's first stage converted here is never published
@@ -1103,6 +1255,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             const int M = e.M;
             const int b = pi % NB;
             uint8_t *pb = parts + b * lay.parts;
+            if constexpr (FMT == 2) {
             if (M == 1) {
                 // ---- integer engine, one token: one accumulator per digit
                 // position j (A = digits * 4^j, one AND per register) ----
@@ -1338,6 +1491,277 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     }
                 }
             }
+            } else {
+            if (M == 1) {
+                // ---- base-3 integer engine, one token: positions p = 0..4 (the
+                // bytes, then their quotients by 3, 9, 27, 81) share one
+                // accumulator; B carries each position's activations ----
+                int acc[2][4];  // [tile][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0;
+                int64_t qsum = 0;
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    qsum += reinterpret_cast<const int64_t *>(sb)[0];
+                    const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        // [tile][row g / g + 8][word 2pr / 2pr + 1]: A words, and their
+                        // even / odd bytes in 16-bit lanes
+                        uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
+                                    E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
+                                    O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
+                                }
+#pragma unroll
+                        for (int p = 0; p < 5; ++p) {
+                            if (p > 0) {
+#pragma unroll
+                                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                                    for (int r = 0; r < 2; ++r)
+#pragma unroll
+                                        for (int h = 0; h < 2; ++h) {
+                                            const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
+                                            const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
+                                            P[t][r][h] = prmt(tE, tO, 0x7351u);
+                                            E[t][r][h] = prmt(tE, 0u, 0x4341u);
+                                            O[t][r][h] = prmt(tO, 0u, 0x4341u);
+                                        }
+                            }
+                            const uint2 bq = *reinterpret_cast<const uint2 *>(xg + dk_i3off(0, pr, p, 0, 0));
+#pragma unroll
+                            for (int t = 0; t < 2; ++t)
+                                mma_u8_16832(acc[t], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1], bq.x,
+                                             bq.y);
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                    break;
+                // V = sum_p 256^p S_p - 2^42 S_ones - Q; lane c holds columns 2c,
+                // 2c + 1 (planes, or the ones column at c = 3), and lane 0 of the
+                // quad forms V (modulo 2^64)
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const uint64_t d0 = (uint32_t)acc[t][2 * rr], d1 = (uint32_t)acc[t][2 * rr + 1];
+                        const uint64_t tc = c < 3 ? d0 + (d1 << 8) : d0;
+                        const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
+                        const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
+                        const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
+                        if (c == 0) {
+                            uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 42);
+                            if (qv == 0) v64 -= (uint64_t)qsum;
+                            reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] = (int64_t)v64;
+                        }
+                    }
+                }
+            } else if (M == 2) {
+                // ---- base-3 integer engine, two tokens: two column groups ----
+                int iacc[2][2][4];  // [tile][column group][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
+                int64_t qsum0 = 0, qsum1 = 0;
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
+                    qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
+                    const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
+#pragma unroll
+                    for (int pr = 0; pr < 2; ++pr) {
+                        uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
+                                    E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
+                                    O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
+                                }
+#pragma unroll
+                        for (int p = 0; p < 5; ++p) {
+                            if (p > 0) {
+#pragma unroll
+                                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                                    for (int r = 0; r < 2; ++r)
+#pragma unroll
+                                        for (int h = 0; h < 2; ++h) {
+                                            const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
+                                            const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
+                                            P[t][r][h] = prmt(tE, tO, 0x7351u);
+                                            E[t][r][h] = prmt(tE, 0u, 0x4341u);
+                                            O[t][r][h] = prmt(tO, 0u, 0x4341u);
+                                        }
+                            }
+                            const uint32_t off = dk_i3off(0, pr, p, 0, 0);
+                            const uint2 bq0 = *reinterpret_cast<const uint2 *>(xg + off);
+                            const uint2 bq1 = *reinterpret_cast<const uint2 *>(xg + 5 * 1024 + off);
+#pragma unroll
+                            for (int t = 0; t < 2; ++t) {
+                                mma_u8_16832(iacc[t][0], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
+                                             bq0.x, bq0.y);
+                                mma_u8_16832(iacc[t][1], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
+                                             bq1.x, bq1.y);
+                            }
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                    break;
+                // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
+                // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+#pragma unroll
+                    for (int rr = 0; rr < 2; ++rr) {
+                        const int64_t d0 = (uint32_t)iacc[t][0][2 * rr], d1 = (uint32_t)iacc[t][0][2 * rr + 1];
+                        const int64_t e0 = (uint32_t)iacc[t][1][2 * rr], e1 = (uint32_t)iacc[t][1][2 * rr + 1];
+                        int64_t v0 = 0, v1 = 0;
+                        if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
+                        else v1 = d0 + (d1 << 8);
+                        if (c < 2) {
+                            v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
+                        } else if (c == 2) {
+                            v0 -= e0 << 42;
+                            v1 -= e0 << 42;
+                        }
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+                        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+                        if (qv == 0) {
+                            v0 -= qsum0;
+                            v1 -= qsum1;
+                        }
+                        if (c == 0) {
+                            int64_t *p = reinterpret_cast<int64_t *>(pb);
+                            p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                            p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
+                        }
+                    }
+                }
+            } else {
+                // ---- base-3 fp16 engine: digits as subnormal halves d 2^-24 in
+                // 16-bit lanes (even bytes, odd bytes), one accumulator ----
+                const int Mp = M + (M & 1);
+                float facc[2][4];  // [tile][D]
+#pragma unroll
+                for (int t = 0; t < 2; ++t) facc[t][0] = facc[t][1] = facc[t][2] = facc[t][3] = 0.f;
+                float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
+                for (int s = e.s0; s < e.s1; ++s) {
+                    const int slot = cs;
+                    if (!wait_stage(slot)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                    const uint8_t *sb = sslot + slot * lay.slot_b;
+                    const float *mt = reinterpret_cast<const float *>(sb);
+                    if (2 * c < M) sx0 += mt[2 * c];
+                    if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
+                    const uint8_t *xb = sb + kDkMetaBytes;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint32_t E[2][2], O[2][2];  // [tile][row g / g + 8]
+#pragma unroll
+                        for (int t = 0; t < 2; ++t)
+#pragma unroll
+                            for (int r = 0; r < 2; ++r) {
+                                const uint32_t W = dk_word(A[t][r], i);
+                                E[t][r] = prmt(W, 0u, 0x4240u);
+                                O[t][r] = prmt(W, 0u, 0x4341u);
+                            }
+#pragma unroll
+                        for (int p = 0; p < 5; ++p) {
+                            uint2 bq = make_uint2(0u, 0u);
+                            if (g < M) bq = *reinterpret_cast<const uint2 *>(xb + dk_h3off(v, i, p, g, c, Mp));
+                            uint32_t dE[2][2], dO[2][2];
+#pragma unroll
+                            for (int t = 0; t < 2; ++t)
+#pragma unroll
+                                for (int r = 0; r < 2; ++r) {
+                                    if (p < 4) {
+                                        // d_p = q_p - 3 q_{p+1} per lane (never negative)
+                                        const uint32_t e1 = prmt(E[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
+                                        const uint32_t o1 = prmt(O[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
+                                        dE[t][r] = E[t][r] - 3u * e1;
+                                        dO[t][r] = O[t][r] - 3u * o1;
+                                        E[t][r] = e1;
+                                        O[t][r] = o1;
+                                    } else {
+                                        dE[t][r] = E[t][r];
+                                        dO[t][r] = O[t][r];
+                                    }
+                                }
+#pragma unroll
+                            for (int t = 0; t < 2; ++t)
+                                mma_16816(facc[t], dE[t][0], dE[t][1], dO[t][0], dO[t][1], bq.x, bq.y);
+                        }
+                    }
+                    release(slot);
+                }
+                if (!ok) break;
+                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                    break;
+                float *p = reinterpret_cast<float *>(pb);
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    float sv[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) sv[q] = facc[t][q] * 16777216.0f;
+                    if (qv == 0) {
+                        sv[0] -= sx0;
+                        sv[1] -= sx1;
+                        sv[2] -= sx0;
+                        sv[3] -= sx1;
+                    }
+                    const int m0 = 2 * c, m1 = 2 * c + 1;
+                    if (m0 < M) {
+                        p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
+                        p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
+                    }
+                    if (m1 < M) {
+                        p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
+                        p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
+                    }
+                }
+            }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[b]);
             ++pi;
@@ -1365,9 +1789,10 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
 // ---- host side ---------------------------------------------------------------
 namespace tlk {
 
-// Relative cost of a stage: the fp16 engine (M >= 3) takes about twice as
-// long per stage as the integer engine.
-inline int dk_stage_cost(int M) { return M <= kDkImmaMaxM ? 1 : 2; }
+// Relative cost of a stage: the fp16 engine (M >= 3) takes about twice (2-bit)
+// or three times (base 3, whose digits take a division each) as long per
+// stage as the integer engine.
+inline int dk_stage_cost(int fmt, int M) { return M <= kDkImmaMaxM ? 1 : (fmt == 2 ? 2 : 3); }
 // Cost per item for a batch of total cost `total` (in integer-engine stages):
 // about four items per SM of a B200, so that the longest-first order leaves a
 // short tail, but 4..16 integer-engine stages of cost, so item boundaries
@@ -1404,21 +1829,25 @@ struct DkSchedule {
     size_t bytes = 0;
 };
 
+// Packed bytes of a row of K trits: 4 (2-bit) or 5 (1.6-bit) trits per byte.
+inline int64_t dk_row_bytes(int fmt, int64_t K) { return fmt == 2 ? (K + 3) / 4 : (K + 4) / 5; }
+
 // Sizes of a batch; with `items` and `units` given, also their tables, holding
 // pointers into the workspace at `ws`.  Items are in layer order, then tile,
 // then part (longest first when no layer reads an earlier one); units in
 // layer order, then stage, then token.
-inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
+inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t *ws,
                               std::vector<DkItemRec> *items, std::vector<DkUnitRec> *units) {
     DkSchedule sc;
     sc.count = count;
-    auto stages_of = [](const DkHostLayer &h) {
-        return (int)((((int64_t)h.K + 3) / 4 + kDkStageW - 1) / kDkStageW);
+    auto stages_of = [fmt](const DkHostLayer &h) {
+        return (int)((dk_row_bytes(fmt, h.K) + kDkStageW - 1) / kDkStageW);
     };
+    auto stage_cost = [fmt](int M) { return dk_stage_cost(fmt, M); };
     int64_t total = 0;
     for (int l = 0; l < count; ++l)
         total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows) *
-                 dk_stage_cost(in[l].M);
+                 stage_cost(in[l].M);
     const int cost = dk_item_cost(total);
     // fp16-engine items stay at 8 stages or more: their epilogue (M outputs
     // per row) must keep up with the consumers.  A layer that waits for the
@@ -1432,7 +1861,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
             const int min_t = (stages_of(h) + (h.M > kDkImmaMaxM ? 1 : 7)) / (h.M > kDkImmaMaxM ? 2 : 8);
             return t > min_t ? t : (min_t > 0 ? min_t : 1);
         }
-        const int t = cost / dk_stage_cost(h.M);
+        const int t = cost / stage_cost(h.M);
         return h.M > kDkImmaMaxM && t < 8 ? 8 : t;
     };
     // An independent layer whose X (pointer, stride, K, M) is an earlier
@@ -1461,7 +1890,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
             if (h.swiglu) sc.chained = 2;
         } else if (src[l] == l) {
             sc.total_units += stages * h.M;
-            sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(h.M));
+            sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(fmt, h.M));
         }
         if (parts > 1) sc.slots += (int64_t)tiles * parts * kDkRows * h.M;
         if (h.M > sc.maxM) sc.maxM = h.M;
@@ -1477,7 +1906,7 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
         const int stages = stages_of(h);
         const int parts = dk_parts(stages, target_of(h));
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
-        const int bstride = kDkMetaBytes + (int)dk_stage_b(h.M);
+        const int bstride = kDkMetaBytes + (int)dk_stage_b(fmt, h.M);
         const bool converts = !h.reads_earlier && src[l] == l;
         uint8_t *B = h.reads_earlier ? nullptr : (converts ? ws + wl.staged + staged : Bs[src[l]]);
         Bs[l] = B;
@@ -1530,9 +1959,9 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
     // the finish its tile may need (one round of loads per token and per
     // four parts, about a stage each), so split tiles finish early.
     if (!sc.chained) {
-        std::stable_sort(items->begin(), items->end(), [](const DkItemRec &x, const DkItemRec &y) {
-            auto cost = [](const DkItemRec &r) {
-                return (r.s1 - r.s0) * dk_stage_cost(r.M) + (r.parts > 1 ? r.M * ((r.parts + 3) / 4) : 0);
+        std::stable_sort(items->begin(), items->end(), [&](const DkItemRec &x, const DkItemRec &y) {
+            auto cost = [&](const DkItemRec &r) {
+                return (r.s1 - r.s0) * stage_cost(r.M) + (r.parts > 1 ? r.M * ((r.parts + 3) / 4) : 0);
             };
             return cost(x) > cost(y);
         });
@@ -1569,10 +1998,10 @@ inline DkSchedule dk_schedule(int count, const DkHostLayer *in, uint8_t *ws,
 
 // Tensor map of a layer's packed weights: bytes x rows, boxes of 128 bytes x
 // 256 rows with the 128-byte swizzle, zero fill outside [0, row bytes) x [0, N).
-inline bool dk_encode_map(const DkHostLayer &h, CUtensorMap *map) {
+inline bool dk_encode_map(int fmt, const DkHostLayer &h, CUtensorMap *map) {
     auto encode = tensor_map_encoder();
     if (!encode) return false;
-    const int64_t rowbytes = ((int64_t)h.K + 3) / 4;
+    const int64_t rowbytes = dk_row_bytes(fmt, h.K);
     cuuint64_t dims[2] = {(cuuint64_t)rowbytes, (cuuint64_t)h.N};
     cuuint64_t strides[1] = {(cuuint64_t)h.ldp};
     cuuint32_t box[2] = {(cuuint32_t)kDkStageW, (cuuint32_t)kDkRows};
@@ -1606,6 +2035,7 @@ inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int
     return a;
 }
 
+template <int FMT>
 inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t stream,
                           int *last_cuda_error) {
     constexpr int kMaxDev = 64;
@@ -1620,14 +2050,14 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     std::call_once(once[dev], [dev] {
         uint32_t most = 0;
         for (int m = 1; m <= 8; ++m) {
-            const uint32_t t = DkLayout(m).total;
+            const uint32_t t = DkLayout(FMT, m).total;
             most = t > most ? t : most;
         }
-        attr_err[dev] = cudaFuncSetAttribute(decode2_kernel<false>,
+        attr_err[dev] = cudaFuncSetAttribute(decode2_kernel<FMT, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
         if (attr_err[dev] == cudaSuccess)
             attr_err[dev] = cudaFuncSetAttribute(
-                decode2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+                decode2_kernel<FMT, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
     });
     if (attr_err[dev] != cudaSuccess) {
         *last_cuda_error = (int)attr_err[dev];
@@ -1636,15 +2066,15 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.total_items < num_sms ? a.total_items : num_sms));
     cfg.blockDim = dim3(kDkThreads);
-    cfg.dynamicSmemBytes = DkLayout(a.maxM).total;
+    cfg.dynamicSmemBytes = DkLayout(FMT, a.maxM).total;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     at[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
     cfg.numAttrs = pdl ? 1 : 0;
-    e = a.chained == 2 ? cudaLaunchKernelEx(&cfg, decode2_kernel<true>, a)
-                       : cudaLaunchKernelEx(&cfg, decode2_kernel<false>, a);
+    e = a.chained == 2 ? cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, true>, a)
+                       : cudaLaunchKernelEx(&cfg, decode2_kernel<FMT, false>, a);
     if (e != cudaSuccess) (void)cudaGetLastError();  // the error is returned here, once
     if (e != cudaSuccess) {
         *last_cuda_error = (int)e;

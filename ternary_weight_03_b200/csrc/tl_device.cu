@@ -12,7 +12,6 @@
 #include "tl_gemv.cuh"
 #include "tl_gemm.cuh"
 #include "tl_gemv3.cuh"
-#include "tl_gemvp.cuh"
 #include "tl_decode.cuh"
 #include "tl_ternarise.cuh"
 
@@ -94,7 +93,7 @@ int check_layer_args(int fmt, const uint8_t *dT, int64_t ldp, const uint16_t *dX
 }
 
 // Validates a batch and converts it into the persistent kernel's host layers.
-int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::GpHostLayer *out) {
+int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::DkHostLayer *out) {
     if (fmt != TL_FMT_2BIT && fmt != TL_FMT_1P6BIT) return TL_ERR_INVALID_ARG;
     if (count < 1 || count > TL_GEMV_BATCH_MAX || !layers) return TL_ERR_INVALID_ARG;
     int64_t items = 0;
@@ -112,41 +111,29 @@ int batch_layers(int fmt, int count, const tl_gemv_layer *layers, tlk::GpHostLay
             // X rows hold [gate | up]: 2K elements, the up half 16-byte aligned
             if (a.ldx < 2 * a.K) return TL_ERR_INVALID_ARG;
             if (a.K % 8 != 0) return TL_ERR_ALIGN;
-            if (fmt != TL_FMT_2BIT) return TL_ERR_UNSUPPORTED;
         }
         if (a.ldx > INT32_MAX || a.ldy > INT32_MAX) return TL_ERR_INVALID_ARG;
-        const int64_t groups = (tl_packed_row_bytes(fmt, a.K) + 63) / 64;
-        items += ((a.N + tlk::kGpRows - 1) / tlk::kGpRows) * groups;  // upper bound
+        const int64_t stages = (tl_packed_row_bytes(fmt, a.K) + tlk::kDkStageW - 1) / tlk::kDkStageW;
+        items += ((a.N + tlk::kDkRows - 1) / tlk::kDkRows) * stages;  // upper bound
         if (items > INT32_MAX / 2) return TL_ERR_INVALID_ARG;
-        out[l] = tlk::GpHostLayer{a.dT, a.dX, a.dY, a.ldp, a.ldx, a.ldy, a.alpha, a.M, (int)a.N,
+        out[l] = tlk::DkHostLayer{a.dT, a.dX, a.dY, a.ldp, a.ldx, a.ldy, a.alpha, a.M, (int)a.N,
                                   (int)a.K, (a.flags & TL_LAYER_READS_EARLIER) != 0, swiglu};
     }
     return TL_OK;
 }
 
-// The 2-bit batch kernel's host layers (the same fields).
-std::vector<tlk::DkHostLayer> dk_layers(const std::vector<tlk::GpHostLayer> &h) {
-    std::vector<tlk::DkHostLayer> out(h.size());
-    for (size_t l = 0; l < h.size(); ++l)
-        out[l] = tlk::DkHostLayer{h[l].T, h[l].X, h[l].Y, h[l].ldp, h[l].ldx, h[l].ldy,
-                                  h[l].alpha, h[l].M, h[l].N, h[l].K, h[l].reads_earlier,
-                                  h[l].swiglu};
-    return out;
-}
-
-// tl_gemv_batch_plan for 2-bit layers (tl_decode.cuh): layer table, tensor
-// maps and zeroed counters written into the workspace.
-int plan_decode2(int count, const std::vector<tlk::GpHostLayer> &h, void *dWorkspace,
+// tl_gemv_batch_plan (tl_decode.cuh): layer table, tensor maps and zeroed
+// counters written into the workspace.
+int plan_decode2(int fmt, int count, const std::vector<tlk::DkHostLayer> &dh, void *dWorkspace,
                  size_t workspace_bytes, tl_gemv_plan *plan) {
-    std::vector<tlk::DkHostLayer> dh = dk_layers(h);
     uint8_t *ws = reinterpret_cast<uint8_t *>(dWorkspace);
     std::vector<tlk::DkItemRec> items;
     std::vector<tlk::DkUnitRec> units;
-    const tlk::DkSchedule sc = tlk::dk_schedule(count, dh.data(), ws, &items, &units);
+    const tlk::DkSchedule sc = tlk::dk_schedule(fmt, count, dh.data(), ws, &items, &units);
     if (sc.bytes > workspace_bytes) return TL_ERR_INVALID_ARG;
     std::vector<CUtensorMap> maps(count);
     for (int l = 0; l < count; ++l)
-        if (!tlk::dk_encode_map(dh[l], &maps[l])) return TL_ERR_CUDA;
+        if (!tlk::dk_encode_map(fmt, dh[l], &maps[l])) return TL_ERR_CUDA;
     if (!device_info()) return TL_ERR_CUDA;
     const tlk::DkWsLayout wl(count, sc.total_items, sc.total_units, sc.total_tiles, sc.slots,
                              sc.staged);
@@ -169,7 +156,7 @@ int plan_decode2(int count, const std::vector<tlk::GpHostLayer> &h, void *dWorks
                        cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e);
-    plan->fmt = TL_FMT_2BIT;
+    plan->fmt = fmt;
     plan->count = count;
     plan->max_m = sc.maxM;
     plan->total_items = sc.total_items;
@@ -263,16 +250,10 @@ int tl_ternarise(int fmt, const uint16_t *dW, int64_t ldw, int64_t N, int64_t K,
 
 int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t *bytes) {
     if (!bytes) return TL_ERR_INVALID_ARG;
-    std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
+    std::vector<tlk::DkHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
     int rc = batch_layers(fmt, count, layers, h.data());
     if (rc != TL_OK) return rc;
-    if (fmt == TL_FMT_2BIT) {
-        std::vector<tlk::DkHostLayer> dh = dk_layers(h);
-        *bytes = tlk::dk_schedule(count, dh.data(), nullptr, nullptr, nullptr).bytes;
-        return TL_OK;
-    }
-    std::vector<tlk::GpLayer> table(count);
-    *bytes = tlk::gp_schedule(fmt, count, h.data(), table.data()).bytes;
+    *bytes = tlk::dk_schedule(fmt, count, h.data(), nullptr, nullptr, nullptr).bytes;
     return TL_OK;
 }
 
@@ -280,40 +261,10 @@ int tl_gemv_batch_plan(int fmt, int count, const tl_gemv_layer *layers, void *dW
                        size_t workspace_bytes, tl_gemv_plan *plan) {
     if (!plan || !dWorkspace) return TL_ERR_INVALID_ARG;
     if (((uintptr_t)dWorkspace & 255u) != 0) return TL_ERR_ALIGN;
-    std::vector<tlk::GpHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
+    std::vector<tlk::DkHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
     int rc = batch_layers(fmt, count, layers, h.data());
     if (rc != TL_OK) return rc;
-    if (fmt == TL_FMT_2BIT) return plan_decode2(count, h, dWorkspace, workspace_bytes, plan);
-    std::vector<tlk::GpLayer> table(count);
-    const tlk::GpSchedule sc = tlk::gp_schedule(fmt, count, h.data(), table.data());
-    if (sc.bytes > workspace_bytes) return TL_ERR_INVALID_ARG;
-    std::vector<CUtensorMap> maps(count);
-    for (int l = 0; l < count; ++l)
-        if (!tlk::gp_encode_map(fmt, h[l], &maps[l])) return TL_ERR_CUDA;
-    if (!device_info()) return TL_ERR_CUDA;
-    const tlk::GpWsLayout wl(count, sc.total_tiles, sc.floats);
-    uint8_t *ws = reinterpret_cast<uint8_t *>(dWorkspace);
-    cudaError_t e = cudaMemset(ws, 0, wl.layers);  // counters
-    if (e == cudaSuccess)
-        e = cudaMemcpy(ws + wl.layers, table.data(), sizeof(tlk::GpLayer) * count,
-                       cudaMemcpyHostToDevice);
-    if (e == cudaSuccess)
-        e = cudaMemcpy(ws + wl.maps, maps.data(), sizeof(CUtensorMap) * count,
-                       cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemset(ws + wl.tiles, 0, (size_t)sc.total_tiles * 4u);
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) return cuda_fail(e);
-    plan->fmt = fmt;
-    plan->count = count;
-    plan->total_units = 0;
-    plan->chained = 0;
-    plan->max_m = sc.maxM;
-    plan->total_items = sc.total_items;
-    plan->total_tiles = sc.total_tiles;
-    plan->dWorkspace = dWorkspace;
-    plan->workspace_bytes = workspace_bytes;
-    plan->generation = 0;
-    return TL_OK;
+    return plan_decode2(fmt, count, h, dWorkspace, workspace_bytes, plan);
 }
 
 int tl_gemv_batch_plan_static(int fmt, int count, const tl_gemv_layer *layers,
@@ -369,20 +320,14 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
             return TL_ERR_INVALID_ARG;
     }
     const bool pdl = (flags & TL_FLAG_PDL) != 0;
-    if (plan->fmt == TL_FMT_2BIT) {
-        tlk::DkArgs da =
-            tlk::dk_args(plan->dWorkspace, plan->count, plan->total_items, plan->total_units,
-                         plan->total_tiles, plan->max_m, plan->chained);
-        da.drop_arrive = (flags & TL_FLAG_DEBUG_DROP_ARRIVE) ? 1 : 0;
-        return tlk::launch_decode2(da, dev->num_sms, pdl, (cudaStream_t)stream, &t_last_cuda_error);
-    }
-    const tlk::GpArgs a = tlk::gp_args(plan->dWorkspace, plan->count, plan->total_items,
-                                       plan->total_tiles, plan->max_m);
+    tlk::DkArgs da = tlk::dk_args(plan->dWorkspace, plan->count, plan->total_items,
+                                  plan->total_units, plan->total_tiles, plan->max_m, plan->chained);
+    da.drop_arrive = (flags & TL_FLAG_DEBUG_DROP_ARRIVE) ? 1 : 0;
     return plan->fmt == TL_FMT_2BIT
-               ? tlk::launch_gemvp<2>(a, dev->num_sms, pdl, (cudaStream_t)stream,
-                                      &t_last_cuda_error)
-               : tlk::launch_gemvp<16>(a, dev->num_sms, pdl, (cudaStream_t)stream,
-                                       &t_last_cuda_error);
+               ? tlk::launch_decode2<2>(da, dev->num_sms, pdl, (cudaStream_t)stream,
+                                        &t_last_cuda_error)
+               : tlk::launch_decode2<16>(da, dev->num_sms, pdl, (cudaStream_t)stream,
+                                         &t_last_cuda_error);
 }
 
 int tl_device_status(void *stream) {

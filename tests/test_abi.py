@@ -129,21 +129,25 @@ def _up(v):
     return (v + 255) // 256 * 256
 
 
-def _ws2_expected(layers):
-    """2-bit batch workspace, region by region (each rounded up to 256 bytes):
+def _ws_expected(layers, fmt=2):
+    """Batch workspace, region by region (each rounded up to 256 bytes):
     counters, one 128-byte tensor map per layer, a 96-byte record per work item
-    (256-row tile x K-part of 2..16 stages of 512 trits), a 48-byte record per
-    conversion unit (stage x token of a layer that reads no earlier output), a
-    u32 per tile, three u32 per layer (ready units, final tiles, tiles), 8-byte
-    partials of split tiles, and the
-    converted activations (64 + 4 KB, 8 KB or 1 KB x even(M) bytes per stage).
-    A layer with a dependency has its items sized to spread it over about
-    148 CTAs (at most 8 parts per tile, 2 for M > 2).  Independent
-    layers with the same X (pointer, ldx, K, M) share the first one's
-    conversion (no units or converted activations of their own)."""
+    (256-row tile x K-part of 2..16 stages of 128 packed bytes per row: 512
+    trits at 2 bits, 640 at 1.6 bits), a 48-byte record per conversion unit
+    (stage x token of a layer that reads no earlier output), a u32 per tile,
+    three u32 per layer (ready units, final tiles, tiles), 8-byte partials of
+    split tiles, and the converted activations (per stage 64 bytes plus one
+    byte per trit and column of 8 per token (M = 1, 2) or two bytes per trit
+    and token rounded up to even (M >= 3)).  A layer with a dependency has its
+    items sized to spread it over about 148 CTAs (at most 8 parts per tile, 2
+    for M > 2).  Independent layers with the same X (pointer, ldx, K, M) share
+    the first one's conversion (no units or converted activations of their
+    own)."""
     items = units = tiles = slots = staged = 0
-    stg = lambda d: -(-(-(-d["K"] // 4)) // 128)
-    cm = lambda d: 1 if d["M"] <= 2 else 2  # relative cost of a stage
+    g = 4 if fmt == 2 else 5  # trits per byte
+    stg = lambda d: -(-(-(-d["K"] // g)) // 128)
+    # relative cost of a stage: fp16 engine x2 (2-bit) or x3 (base 3)
+    cm = lambda d: 1 if d["M"] <= 2 else (2 if fmt == 2 else 3)
     total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
     cost = min(16, max(4, total // (4 * 148)))  # cost per item
     seen = set()
@@ -165,7 +169,7 @@ def _ws2_expected(layers):
         if not d.get("flags", 0) and key not in seen:
             seen.add(key)
             units += stages * d["M"]
-            b = 4096 if d["M"] == 1 else (8192 if d["M"] == 2 else 1024 * (d["M"] + d["M"] % 2))
+            b = 8 * 128 * g * d["M"] if d["M"] <= 2 else 2 * 128 * g * (d["M"] + d["M"] % 2)
             staged += stages * (64 + b)
         if parts > 1:
             slots += t * parts * 256 * d["M"]
@@ -189,16 +193,13 @@ def test_batch_workspace_size(L):
              [dict(base, N=3072, K=3072, M=2)] * 3 + [dict(base, N=3072, K=3072, M=2, dX=A + 65536)]
              + [dict(base, N=8192, K=3072, M=2, dX=A + 131072)] * 2
              + [dict(base, N=3072, K=8192, M=2, flags=3, ldx=16384)]]
-    for ls in cases:
-        arr = _layers([dict(d, ldp=(d["K"] + 3) // 4 + (-((d["K"] + 3) // 4)) % 16,
-                            ldx=d.get("ldx", d["K"] + (-d["K"]) % 8),
-                            ldy=d["N"] + (-d["N"]) % 8) for d in ls])
-        rc, n = _ws(L, 2, arr)
-        assert rc == 0 and n == _ws2_expected(ls), (ls, n)
-    # 1.6-bit: table (one 88-byte entry + one 128-byte TMA descriptor per layer),
-    # counters, and fp32 partials only for layers whose rows are split
-    rc, n = _ws(L, 16, _layers([dict(N=1000, K=2048, ldp=416, ldx=2048, ldy=1000)]))
-    assert rc == 0 and n == 1024  # header 256, table 256, map 256, 9 tile counters 256
+    for fmt, g in ((2, 4), (16, 5)):
+        for ls in cases:
+            arr = _layers([dict(d, ldp=(d["K"] + g - 1) // g + (-((d["K"] + g - 1) // g)) % 16,
+                                ldx=d.get("ldx", d["K"] + (-d["K"]) % 8),
+                                ldy=d["N"] + (-d["N"]) % 8) for d in ls])
+            rc, n = _ws(L, fmt, arr)
+            assert rc == 0 and n == _ws_expected(ls, fmt), (fmt, ls, n)
 
 
 @pytest.mark.parametrize("spec,count,rc", [
@@ -221,7 +222,8 @@ def test_batch_argument_rules(L, spec, count, rc):
     (2, dict(flags=3, ldx=1024), 1),                 # rows shorter than 2K
     (2, dict(flags=3, K=1020, ldx=2048, ldp=256), 4),  # up half not 16-byte aligned
     (2, dict(flags=4), 1),                           # unknown flag
-    (16, dict(flags=3, ldx=2048), 7),                # 1.6-bit batch: unsupported
+    (16, dict(flags=3, ldx=2048), 0),                # 1.6-bit batch too
+    (16, dict(flags=3, ldx=1024), 1),
 ])
 def test_swiglu_input_rules(L, fmt, second, rc):
     import ctypes

@@ -287,7 +287,7 @@ def test_long_chain_multiple_items_per_cta(fmt):
 DECODE_LAYER = [(3072, 3072)] * 4 + [(3072, 8192)] * 2 + [(8192, 3072)]  # q k v o gate up down
 
 
-@pytest.mark.parametrize("fmt,M", [(2, 1), (2, 8), (16, 1)])
+@pytest.mark.parametrize("fmt,M", [(2, 1), (2, 8), (16, 1), (16, 2), (16, 8)])
 def test_decode_step_210_layers_sampled(fmt, M):
     """The 30-layer decode step (210 matrices, 849 MB packed at 2 bits) as ONE
     batch launch, the configuration the bench times; per layer, sampled
@@ -328,8 +328,9 @@ def _silu_glu(gu, F):
     return g / (1.0 + np.exp(-g)) * u
 
 
+@pytest.mark.parametrize("fmt", [2, 16])
 @pytest.mark.parametrize("M", [1, 2, 3, 8])
-def test_swiglu_down_projection(M):
+def test_swiglu_down_projection(fmt, M):
     """Gate and up projections write the two halves of one buffer; the down
     projection reads it with TL_LAYER_SWIGLU_INPUT, its input formed on chip
     as fp16(silu(g) * u).  Checked layer by layer against the oracle: gate
@@ -349,12 +350,12 @@ def test_swiglu_down_projection(M):
     GU = torch.full((M, 2 * F), float("nan"), dtype=torch.float16, device="cuda")
     Yx = torch.full((M, 504), float("nan"), dtype=torch.float16, device="cuda")
     Yd = torch.full((M, H2 + (-H2) % 8), float("nan"), dtype=torch.float16, device="cuda")
-    pk = lambda T: torch.from_numpy(tl.pack(2, T)).cuda()
+    pk = lambda T: torch.from_numpy(tl.pack(fmt, T)).cuda()
     specs = [(pk(Tg), ag, dX0, H, GU[:, :F]), (pk(Tu), au, dX0, H, GU[:, F:]),
              (pk(Tx), ax, dX0, H, Yx),
              (pk(Td), ad, GU, F, Yd, tl.LAYER_READS_EARLIER | tl.LAYER_SWIGLU_INPUT)]
-    layers = tl.make_layers(2, specs)
-    plan, ws = _plan(2, layers)
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
     outs = []
     for _ in range(2):
         Yd.fill_(float("nan"))
@@ -376,8 +377,9 @@ def test_swiglu_down_projection(M):
     assert np.isnan(Yd[:, H2:].float().cpu().numpy()).all(), "wrote past column N"
 
 
+@pytest.mark.parametrize("fmt", [2, 16])
 @pytest.mark.parametrize("M", [1, 8])
-def test_layers_sharing_x(M):
+def test_layers_sharing_x(fmt, M):
     """Q, K and V on one X (one conversion of X, three alphas), O on another
     X, and two layers on a third: each layer against the oracle, and the
     batch needs less workspace than the same layers on distinct X copies."""
@@ -392,15 +394,15 @@ def test_layers_sharing_x(M):
     cases, specs, specs_copy = [], [], []
     for i, (N, a, xi) in enumerate(shapes):
         T = synth.trits(95 + i, N, K)
-        dP = torch.from_numpy(tl.pack(2, T)).cuda()
+        dP = torch.from_numpy(tl.pack(fmt, T)).cuda()
         dY = torch.full((M + 1, N + (-N) % 8), float("nan"), dtype=torch.float16, device="cuda")
         specs.append((dP, a, xs[xi][1], K, dY[:M]))
         specs_copy.append((dP, a, xs[xi][1].clone(), K, dY[:M]))
         cases.append((T, xs[xi][0], a, dY, N))  # row M is a guard row
-    layers = tl.make_layers(2, specs)
-    shared_bytes = tl.gemv_batch_bytes(2, layers)
-    assert shared_bytes < tl.gemv_batch_bytes(2, tl.make_layers(2, specs_copy))
-    plan, ws = _plan(2, layers)
+    layers = tl.make_layers(fmt, specs)
+    shared_bytes = tl.gemv_batch_bytes(fmt, layers)
+    assert shared_bytes < tl.gemv_batch_bytes(fmt, tl.make_layers(fmt, specs_copy))
+    plan, ws = _plan(fmt, layers)
     tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
     assert tl.device_status() == 0
     for T, X, a, dY, N in cases:
