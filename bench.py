@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -454,8 +455,10 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
     distinct seeded matrices (p0 = 1/3, alpha ~ U(0.01, 0.05)), each with its
     own seeded activation vector(s), run as ONE tl_gemv_batch_run per step
     (graph-captured, programmatic dependent launch).  "chained" reruns the
-    2-bit M = 1 step with every layer flagged as reading the earlier layers'
-    outputs (a serial dependency per layer).  "fused" (2-bit) runs the step
+    2-bit M = 1 step as one chain: layer i reads (the first K_i columns of)
+    the buffer whose first N_{i-1} columns layer i - 1 writes, flagged
+    TL_LAYER_READS_EARLIER (a serial dependency per layer; alpha =
+    1 / sqrt(2K/3) keeps the chained values in range).  "fused" (2-bit) runs the step
     as a decoder would: q, k and v on one shared X (converted once), gate
     and up on another, writing the two halves of one buffer, and down
     reading silu(gate) * up from it (TL_LAYER_SWIGLU_INPUT, a dependency on
@@ -504,8 +507,19 @@ def decode_step(dev, stream, fmts=(2, 16), ms=(1, 8), steps: int = 20, warmup: i
             variants = [("", 0)] + ([("_chained", tl.LAYER_READS_EARLIER)]
                                     if fmt == 2 and M == 1 else [])
             for suffix, flag in variants:
-                specs = [(dP, alpha, X, K, Y, flag if i else 0)
-                         for i, ((K, N, dP, alpha), X, Y) in enumerate(zip(dev_mats, xs, ys))]
+                if flag:
+                    # buffer i holds layer i's input; layer i - 1 writes its first columns
+                    bufs = []
+                    for i, (K, N, seed) in enumerate(mats):
+                        w = max(K, mats[i - 1][1] if i else 0)
+                        w += (-w) % 8
+                        bufs.append(torch.from_numpy(synth.activations(seed, M, w)).to(dev))
+                    specs = [(dP, 1.0 / math.sqrt(2.0 * K / 3.0), bufs[i][:, :K], K,
+                              bufs[i + 1][:, :N] if i + 1 < len(bufs) else ys[i], flag if i else 0)
+                             for i, (K, N, dP, alpha) in enumerate(dev_mats)]
+                else:
+                    specs = [(dP, alpha, X, K, Y)
+                             for (K, N, dP, alpha), X, Y in zip(dev_mats, xs, ys)]
                 layers = tl.make_layers(fmt, specs)
                 ws = torch.zeros(tl.gemv_batch_bytes(fmt, layers), dtype=torch.uint8, device=dev)
                 plan = tl.gemv_batch_plan(fmt, layers, ws)

@@ -187,10 +187,13 @@ int tl_gemv_batch_bytes(int fmt, int count, const tl_gemv_layer *layers, size_t 
  * into a CUDA graph.  Plan once, run many times; the plan holds the
  * pointers of T, X and Y, so a batch on other buffers needs a new plan.
  * Dependencies: a layer with TL_LAYER_READS_EARLIER (not allowed on layer
- * 0) reads its X only after every earlier layer of the batch has stored its
- * Y, so it may consume their outputs (a chain of layers); without the flag,
- * X must not be written by any layer of the batch.  No Y may overlap another
- * layer's Y, X or T.
+ * 0) may consume the outputs of earlier layers of the batch: it reads its X
+ * only after every earlier layer whose Y overlaps that X (rows m < M of K
+ * elements at stride ldx, 2K with the SwiGLU input; compared by address) has
+ * stored all of its Y.  Layers it does not read from run concurrently with
+ * it, so independent chains (one per decoder block, say) overlap.  Without
+ * the flag, X must not be written by any layer of the batch.  No Y may
+ * overlap another layer's Y or T, nor the X of an earlier layer.
  * SwiGLU input (TL_LAYER_SWIGLU_INPUT together with
  * TL_LAYER_READS_EARLIER): row m of dX holds a gated unit's two inputs, the
  * gate values g in elements [0, K) and the up values u in [K, 2K) (typically

@@ -91,7 +91,6 @@ constexpr uint32_t kDkSmemBudget = 232448u;             // 227 KB
 constexpr int kDkMetaBytes = 64;                        // per stage: per-token offsets, first
 
 // Workspace counters (u32 words of the 256-byte header).
-constexpr int kDkCtrPrefix = 1;     // layers 0 .. prefix - 1 have all their outputs stored
 constexpr int kDkCtrDone = 2;       // CTAs that have finished
 constexpr int kDkCtrItems = 3;      // items handed out beyond the first 2 gridDim.x
 constexpr int kDkCtrUnitsDone = 5;  // CTAs whose conversion units are all written
@@ -131,9 +130,11 @@ struct DkItemRec {
     int M, K, N, ldx, ldy;
     int parts;         // K-parts per tile of the layer
     int tile_begin;    // global index of the layer's first tile
-    int wait_tiles;    // 1: X is read once every earlier layer is complete (0: no wait)
-    int need;          // conversion units of X (stages x M); chained layers: 1 if X
-                       // holds [gate | up] halves (SwiGLU input), else 0
+    int deps;          // 0: X is final at the start; else (lo << 16) | (hi + 1): X is
+                       // read once layers lo .. hi (the earlier layers whose Y overlaps
+                       // it) have stored all their outputs
+    int need;          // conversion units of X (stages x M); layers converted on chip
+                       // (B == null): 1 if X holds [gate | up] halves (SwiGLU input)
     int bstride;       // bytes per stage of B (64 + dk_stage_b(M))
 };
 static_assert(sizeof(DkItemRec) == 96, "item record is six 16-byte loads");
@@ -830,7 +831,6 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         bool wrapped = false;
         int qi = 0;
         bool waited = false, ok = true, all_ready = a.total_units == 0, fenced = true;
-        uint32_t prefix_seen = 0;  // complete layers known to this producer
         const int G = (int)gridDim.x;
         int item = (int)blockIdx.x;
         DkItemRec R{};
@@ -867,8 +867,8 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     e.parts = R.parts;
                     e.tile_begin = R.tile_begin;
                     e.pre = pre ? 1 : 0;
-                    e.chained = R.wait_tiles > 0 ? 1 : 0;
-                    e.swiglu = R.wait_tiles > 0 && (R.need & 1) ? 1 : 0;
+                    e.chained = R.deps != 0 ? 1 : 0;
+                    e.swiglu = R.B == nullptr && (R.need & 1) ? 1 : 0;
                     e.layer = R.layer & 0xFFFF;
                 }
                 queue[q] = e;
@@ -898,11 +898,11 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                                              &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
                         fenced = false;
                     }
-                } else if (R.wait_tiles > 0 && prefix_seen < (uint32_t)(R.layer & 0xFFFF)) {
-                    // every earlier layer complete: the prefix reaches this layer
-                    good = dk_wait_count(&a.ctr[kDkCtrPrefix], (uint32_t)(R.layer & 0xFFFF), nullptr, 0u,
-                                         nullptr);
-                    if (good) prefix_seen = (uint32_t)(R.layer & 0xFFFF);
+                } else if (R.deps != 0) {
+                    // every layer that writes this layer's X has stored all its tiles
+                    const int hi = (R.deps & 0xFFFF) - 1;
+                    for (int j = R.deps >> 16; j <= hi && good; ++j)
+                        good = dk_wait_count(&a.lfinal[j], a.ltiles[j], nullptr, 0u, nullptr);
                     fenced = false;
                 }
                 // what was observed above is read next by bulk copies (async proxy)
@@ -932,7 +932,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 // counter, which the previous grid's last CTA reset
                 next = item + G;
                 const bool in_ok = wait_inputs();
-                if (lane == 0 && in_ok && R.wait_tiles > 0) {
+                if (lane == 0 && in_ok && R.deps != 0) {
                     __threadfence_block();
                     iready[q] = item;  // the stagers may convert this item's X
                 }
@@ -958,7 +958,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     break;
                 }
             } else {
-                if (R.wait_tiles > 0) {
+                if (R.deps != 0) {
                     // a dependent item: its weights do not depend on the earlier
                     // layers, so up to a ring's worth streams while it waits (the
                     // slots are freed by earlier items, never by this one)
@@ -986,7 +986,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     ok = false;
                     break;
                 }
-                if (lane == 0 && R.wait_tiles > 0) {
+                if (lane == 0 && R.deps != 0) {
                     __threadfence_block();
                     iready[q] = item;  // the stagers may convert this item's X
                 }
@@ -1201,21 +1201,12 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 }
             }
             if (final_tile && a.chained) {
-                // the tile's outputs are stored: count it for its layer; the last
-                // tile of a layer advances the prefix of complete layers as far as
-                // it goes (whoever completes the next layer continues), so a
-                // dependent layer waits for every earlier layer, however the
-                // layers' tiles interleave
+                // the tile's outputs are stored: count it for its layer (a layer
+                // whose count reaches its tiles is complete for its readers)
                 dk_fence_proxy_global();
                 __threadfence();
                 __syncwarp();
-                if (lane == 0 && atomicAdd(&a.lfinal[e.layer], 1u) == a.ltiles[e.layer] - 1u) {
-                    for (int guard = 0; guard <= a.count; ++guard) {
-                        const uint32_t p = dk_ld_acquire(&a.ctr[kDkCtrPrefix]);
-                        if (p >= (uint32_t)a.count || dk_ld_acquire(&a.lfinal[p]) < a.ltiles[p]) break;
-                        atomicCAS(&a.ctr[kDkCtrPrefix], p, p + 1u);
-                    }
-                }
+                if (lane == 0) atomicAdd(&a.lfinal[e.layer], 1u);
             }
         }
     } else {
@@ -1775,7 +1766,6 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         const uint32_t done = atomicAdd(&a.ctr[kDkCtrDone], 1u);
         if (done == gridDim.x - 1) {
             __threadfence();
-            a.ctr[kDkCtrPrefix] = 0u;
             a.ctr[kDkCtrItems] = 0u;
             a.ctr[kDkCtrUnitsDone] = 0u;
             for (int l = 0; l < a.count; ++l) a.ready[l] = a.lfinal[l] = 0u;
@@ -1878,6 +1868,26 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
                 break;
             }
     }
+    // The earlier layers whose Y overlaps a dependent layer's X (its rows of K,
+    // or 2K with the SwiGLU input, elements): deps[l] = (lo << 16) | (hi + 1)
+    // for the first and last of them, 0 if none (X is then final at the start).
+    std::vector<int> deps(count, 0);
+    for (int l = 0; l < count; ++l) {
+        if (!in[l].reads_earlier) continue;
+        const DkHostLayer &h = in[l];
+        const uint8_t *x0 = reinterpret_cast<const uint8_t *>(h.X);
+        const uint8_t *x1 = x0 + 2 * ((int64_t)(h.M - 1) * h.ldx + (h.swiglu ? 2 * (int64_t)h.K : h.K));
+        int lo = -1, hi = -1;
+        for (int j = 0; j < l; ++j) {
+            const uint8_t *y0 = reinterpret_cast<const uint8_t *>(in[j].Y);
+            const uint8_t *y1 = y0 + 2 * ((int64_t)(in[j].M - 1) * in[j].ldy + in[j].N);
+            if (y0 < x1 && x0 < y1) {
+                if (lo < 0) lo = j;
+                hi = j;
+            }
+        }
+        if (lo >= 0) deps[l] = (lo << 16) | (hi + 1);
+    }
     for (int l = 0; l < count; ++l) {
         const DkHostLayer &h = in[l];
         const int stages = stages_of(h);
@@ -1930,7 +1940,7 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
                 r.ldy = (int)h.ldy;
                 r.parts = parts;
                 r.tile_begin = tile_begin;
-                r.wait_tiles = h.reads_earlier ? 1 : 0;
+                r.deps = deps[l];
                 r.need = h.reads_earlier ? (h.swiglu ? 1 : 0) : stages * h.M;
                 r.bstride = bstride;
                 items->push_back(r);
@@ -1968,8 +1978,8 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
         return sc;
     }
     // With dependencies, a dependent layer's items must follow every item of
-    // the earlier layers (then everything it waits for was handed out before
-    // it).  Within that rule, each dependent layer's items are handed out
+    // the layers it reads (then everything it waits for was handed out before
+    // it); they follow every earlier layer's.  Within that rule, each dependent layer's items are handed out
     // after the independent layers that follow it, just before the next
     // dependent layer's: a CTA that takes a dependent item then mostly finds
     // its inputs complete instead of waiting while independent work remains.
@@ -1981,7 +1991,7 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
         const int layer = (*items)[i].layer & 0xFFFF;
         size_t j = i;
         while (j < items->size() && ((*items)[j].layer & 0xFFFF) == layer) ++j;
-        if ((*items)[i].wait_tiles > 0) {
+        if ((*items)[i].deps != 0) {
             ordered.insert(ordered.end(), items->begin() + pending_begin,
                            items->begin() + pending_end);
             pending_begin = i;

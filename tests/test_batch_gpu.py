@@ -458,3 +458,62 @@ def test_dependent_layer_before_independent_ones(fmt):
     for T, X, Y in small:
         ref = o.linear(T, X, 0.05)
         assert (np.abs(Y.float().cpu().numpy() - ref) <= oracle.tolerance(ref, X, 0.05)).all()
+
+
+@pytest.mark.parametrize("fmt", [2, 16])
+def test_interleaved_chains(fmt):
+    """Dependencies follow the data: a dependent layer waits for the earlier
+    layers whose Y overlaps its X, not for every earlier layer.  Two chains
+    interleave (a0, b0, a1 reads a0, b1 reads b0's output plus 500 more
+    columns of the same buffer), and a flagged SwiGLU layer whose [gate | up]
+    input no layer of the batch writes runs without waiting.  Each layer
+    against the oracle on the inputs as stored; two runs agree bit for bit."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    M, K0 = 2, 3000
+    X0, X1 = synth.activations(130, M, K0), synth.activations(131, M, K0)
+    GUc = synth.activations(132, M, 2 * 800)
+    Ta0, Tb0 = synth.trits(133, 1000, K0), synth.trits(134, 2000, K0)
+    Ta1, Tb1, Tc = synth.trits(135, 700, 1000), synth.trits(136, 900, 2500), synth.trits(137, 600, 800)
+    aa0, ab0, aa1, ab1, ac = 0.02, 0.013, 0.031, 0.017, 0.025
+    dX0, dX1, dGU = (torch.from_numpy(v).cuda() for v in (X0, X1, GUc))
+    bufA = torch.full((M, 1000), float("nan"), dtype=torch.float16, device="cuda")
+    tail = synth.activations(138, M, 500)
+    bufB = torch.full((M, 2504), float("nan"), dtype=torch.float16, device="cuda")
+    bufB[:, 2000:2500] = torch.from_numpy(tail).cuda()
+    Za = torch.full((M, 704), float("nan"), dtype=torch.float16, device="cuda")
+    Zb = torch.full((M, 904), float("nan"), dtype=torch.float16, device="cuda")
+    Zc = torch.full((M, 600), float("nan"), dtype=torch.float16, device="cuda")
+    pk = lambda T: torch.from_numpy(tl.pack(fmt, T)).cuda()
+    RE, SW = tl.LAYER_READS_EARLIER, tl.LAYER_SWIGLU_INPUT
+    specs = [(pk(Ta0), aa0, dX0, K0, bufA), (pk(Tb0), ab0, dX1, K0, bufB[:, :2000]),
+             (pk(Ta1), aa1, bufA, 1000, Za, RE), (pk(Tb1), ab1, bufB[:, :2500], 2500, Zb, RE),
+             (pk(Tc), ac, dGU, 800, Zc, RE | SW)]
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    outs = []
+    for _ in range(2):
+        for z in (Za, Zb, Zc):
+            z.fill_(float("nan"))
+        tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+        assert tl.device_status() == 0
+        outs.append([z.cpu().numpy().view(np.uint16).copy() for z in (Za, Zb, Zc)])
+    assert all(np.array_equal(u, v) for u, v in zip(*outs)), "not deterministic"
+    o = oracle.get()
+
+    def check(T, x, a, got, stored):
+        ref = o.linear(T, x, a, nthreads=8)
+        tol = oracle.tolerance(ref, x, a)
+        if stored:  # x was stored as binary16 by an earlier layer (or rounded once here)
+            tol = tol + abs(a) * np.spacing(np.abs(x).astype(np.float16)).astype(np.float64).sum(axis=1)[:, None]
+        err = np.abs(got.astype(np.float64) - ref)
+        assert (err <= tol).all(), f"{int((err > tol).sum())} of {err.size} outside tolerance"
+
+    A, B = bufA.cpu().numpy(), bufB.cpu().numpy()
+    check(Ta0, X0, aa0, A, False)
+    check(Tb0, X1, ab0, B[:, :2000], False)
+    check(Ta1, A, aa1, Za[:, :700].cpu().numpy(), True)
+    check(Tb1, B[:, :2500], ab1, Zb[:, :900].cpu().numpy(), True)
+    assert np.array_equal(B[:, 2000:2500], tail), "the columns no layer writes changed"
+    x = _silu_glu(GUc, 800).astype(np.float16)
+    check(Tc, x, ac, Zc.cpu().numpy(), True)
