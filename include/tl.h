@@ -164,13 +164,14 @@ typedef struct tl_gemv_plan {
     uint64_t generation; /* 0, or the static plan's number (tl_gemv_batch_plan_static) */
 } tl_gemv_plan;
 
-/* Workspace bytes a batch needs: counters, one TMA descriptor per layer, a
- * 96-byte record per work item (256 output rows x a K-part of whole stages;
+/* Workspace bytes a batch needs: counters (16 bytes per layer), one TMA
+ * descriptor per layer, a 112-byte record per work item (256 output rows x a K-part of whole stages;
  * a stage is 128 packed bytes per row, 512 trits at 2 bits or 640 at 1.6
  * bits), the layers' activations converted once into the tensor-core
  * operand layout (per stage 64 B plus 8 B per trit x M at M <= 2, 2 B per
  * trit x M rounded up to even at M >= 3; none for TL_LAYER_READS_EARLIER
- * layers, which convert on chip) with a 48-byte record per stage and token,
+ * layers with M <= 2, which convert on chip) with a 48-byte record per stage
+ * and token (none for TL_LAYER_READS_EARLIER layers),
  * and 8-byte partial sums of rows split into K-parts (N * M * 8 bytes per
  * part).  Validates the batch like tl_gemv_batch_plan.  Pure host
  * function. */

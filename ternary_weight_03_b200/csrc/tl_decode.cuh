@@ -133,11 +133,18 @@ struct DkItemRec {
     int deps;          // 0: X is final at the start; else (lo << 16) | (hi + 1): X is
                        // read once layers lo .. hi (the earlier layers whose Y overlaps
                        // it) have stored all their outputs
-    int need;          // conversion units of X (stages x M); layers converted on chip
-                       // (B == null): 1 if X holds [gate | up] halves (SwiGLU input)
+    int need;          // conversion units of X (stages x M) when B is given, else 0
     int bstride;       // bytes per stage of B (64 + dk_stage_b(M))
+    int flags;         // kDkItemSwiglu, kDkItemCoop
+    int pad_[3];
 };
-static_assert(sizeof(DkItemRec) == 96, "item record is six 16-byte loads");
+static_assert(sizeof(DkItemRec) == 112, "item record is seven 16-byte loads");
+// DkItemRec.flags: X rows hold [gate | up] halves (SwiGLU input); X is written
+// by earlier layers and converted into B once, after they complete, by the
+// stagers of whichever CTAs hold the layer's items (units claimed from a
+// per-layer counter), instead of on chip by every item.
+constexpr int kDkItemSwiglu = 1;
+constexpr int kDkItemCoop = 2;
 
 // One conversion unit: one stage of one token of one layer.
 struct DkUnitRec {
@@ -154,7 +161,8 @@ static_assert(sizeof(DkUnitRec) == 48, "unit record is three 16-byte loads");
 //   items   : total_items x DkItemRec
 //   units   : total_units x DkUnitRec
 //   ready   : count x u32, conversion units written per layer; then count x u32,
-//             final tiles per layer; then count x u32, tiles per layer
+//             final tiles per layer; count x u32, tiles per layer; count x u32,
+//             conversion units claimed per layer (kDkItemCoop)
 //   tiles   : total_tiles x u32, parts of each tile that have arrived
 //   partials: 8-byte partial sums of split tiles (int64 for M <= 2, double above)
 //   staged  : converted operands, per layer stages x (64 + dk_stage_b(M)) bytes
@@ -167,7 +175,7 @@ struct DkWsLayout {
         items = up(maps + (size_t)count * sizeof(CUtensorMap));
         units = up(items + (size_t)total_items * sizeof(DkItemRec));
         ready = up(units + (size_t)total_units * sizeof(DkUnitRec));
-        tiles = up(ready + (size_t)count * 12u);
+        tiles = up(ready + (size_t)count * 16u);
         partials = up(tiles + (size_t)total_tiles * 4u);
         staged = up(partials + (size_t)slots * 8u);
         total = up(staged + (size_t)staged_bytes);
@@ -182,6 +190,7 @@ struct DkArgs {
     uint32_t *ready;
     uint32_t *lfinal;        // final tiles per layer (batches with dependencies)
     const uint32_t *ltiles;  // tiles per layer
+    uint32_t *claim;         // conversion units claimed per layer (kDkItemCoop)
     uint32_t *tile_ctr;
     int64_t *partials;
     int count;
@@ -203,6 +212,7 @@ struct DkQEntry {
     int chained;  // X is written by earlier layers of this launch
     int swiglu;   // X rows hold [gate | up]; the input is silu(gate) * up
     int layer;    // the item's layer
+    int coop;     // the stagers first help convert the layer's X into B (kDkItemCoop)
 };
 
 struct DkLayout {
@@ -746,6 +756,34 @@ __device__ __noinline__ void dk_finalize(const int64_t *base, int cnt, int parts
 
 // kGlu: the batch has SwiGLU-input layers (a separate instantiation, so that
 // the conversion's fp32 silu code is not part of every other batch's kernel).
+// A dependent layer's X converted once (kDkItemCoop): a warp claims the
+// layer's units (stage, token) one at a time until none is left, converts each
+// into the layer's B in the workspace and counts it in `ready`.  Not inlined,
+// so its registers do not weigh on the kernel's other roles.
+template <int FMT>
+__device__ __noinline__ void dk_coop_convert(const DkItemRec *ir, const uint16_t *X, int ldx, int M,
+                                             int K, bool swiglu, uint32_t *claim, uint32_t *ready,
+                                             int lane) {
+    constexpr int TS = dk_trits(FMT);
+    uint8_t *B = const_cast<uint8_t *>(ir->B);
+    const int need = ir->need, bstride = ir->bstride;
+    while (true) {
+        uint32_t u = 0;
+        if (lane == 0) u = atomicAdd(claim, 1u);
+        u = __shfl_sync(0xffffffffu, u, 0);
+        if (u >= (uint32_t)need) break;
+        const int us = (int)u / M, um = (int)u % M;
+        const int valid = min(K - us * TS, TS);
+        const uint16_t *src = X + (int64_t)um * ldx + (int64_t)us * TS;
+        dk_convert<FMT>(src, swiglu ? src + K : nullptr, valid, um, M, B + (int64_t)us * bstride, lane);
+        // read by bulk copies of other CTAs
+        dk_fence_proxy_global();
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(ready, 1u);
+    }
+}
+
 template <int FMT, bool kGlu>
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
     constexpr int TS = dk_trits(FMT);  // activations per stage
@@ -834,7 +872,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
         const int G = (int)gridDim.x;
         int item = (int)blockIdx.x;
         DkItemRec R{};
-        if (item < a.total_items) R = dk_load_rec<DkItemRec, 6>(a.items, item);
+        if (item < a.total_items) R = dk_load_rec<DkItemRec, 7>(a.items, item);
         int next = a.total_items;
         while (ok) {
             const int q = qi % kDkQueue;
@@ -868,8 +906,9 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     e.tile_begin = R.tile_begin;
                     e.pre = pre ? 1 : 0;
                     e.chained = R.deps != 0 ? 1 : 0;
-                    e.swiglu = R.B == nullptr && (R.need & 1) ? 1 : 0;
+                    e.swiglu = (R.flags & kDkItemSwiglu) ? 1 : 0;
                     e.layer = R.layer & 0xFFFF;
+                    e.coop = (R.flags & kDkItemCoop) ? 1 : 0;
                 }
                 queue[q] = e;
                 mbar_arrive(&qfull[q]);
@@ -888,22 +927,39 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     dk_bulk_load(sslot + slot * lay.slot_b, R.B + (int64_t)s * R.bstride,
                                  (uint32_t)R.bstride, &wfull[slot]);
             };
-            // the item's activations may be read: the layer's units are
-            // converted, or (chained layers) the earlier layers' outputs are final
+            const bool coop = (R.flags & kDkItemCoop) != 0;
+            // the item's activations may be read: the earlier layers that write
+            // X are complete (dependent layers), and the layer's units are
+            // converted (operands that arrive with the weights)
             auto wait_inputs = [&]() -> bool {
                 bool good = true;
-                if (pre) {
-                    if (!all_ready) {
-                        good = dk_wait_count(&a.ready[R.layer >> 16], (uint32_t)R.need,
-                                             &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
-                        fenced = false;
-                    }
-                } else if (R.deps != 0) {
+                if (R.deps != 0) {
                     // every layer that writes this layer's X has stored all its tiles
                     const int hi = (R.deps & 0xFFFF) - 1;
                     for (int j = R.deps >> 16; j <= hi && good; ++j)
                         good = dk_wait_count(&a.lfinal[j], a.ltiles[j], nullptr, 0u, nullptr);
                     fenced = false;
+                }
+                if (good && R.deps != 0) {
+                    // the stagers may read X: to convert the item's stages, or
+                    // (coop) to help convert the layer's units
+                    if (lane == 0) {
+                        __threadfence_block();
+                        iready[q] = item;
+                    }
+                    __syncwarp();
+                }
+                if (good && pre) {
+                    if (coop) {
+                        // units of a dependent layer: converted during this launch
+                        good = dk_wait_count(&a.ready[R.layer & 0xFFFF], (uint32_t)R.need, nullptr, 0u,
+                                             nullptr);
+                        fenced = false;
+                    } else if (!all_ready) {
+                        good = dk_wait_count(&a.ready[R.layer >> 16], (uint32_t)R.need,
+                                             &a.ctr[kDkCtrUnitsDone], gridDim.x, &all_ready);
+                        fenced = false;
+                    }
                 }
                 // what was observed above is read next by bulk copies (async proxy)
                 if (!fenced) {
@@ -932,10 +988,6 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                 // counter, which the previous grid's last CTA reset
                 next = item + G;
                 const bool in_ok = wait_inputs();
-                if (lane == 0 && in_ok && R.deps != 0) {
-                    __threadfence_block();
-                    iready[q] = item;  // the stagers may convert this item's X
-                }
                 if (lane == 0) {
                     for (int i = 0; i < pre_n; ++i) {
                         const int slot = (int)((stage + i) % NS);
@@ -958,11 +1010,14 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                     break;
                 }
             } else {
-                if (R.deps != 0) {
+                int pre_n = 0;
+                const int s_pre = s, ps_pre = ps;
+                if (R.deps != 0 || coop) {
                     // a dependent item: its weights do not depend on the earlier
                     // layers, so up to a ring's worth streams while it waits (the
-                    // slots are freed by earlier items, never by this one)
-                    const int pre_n = min(R.s1 - s, NS);
+                    // slots are freed by earlier items, never by this one); with
+                    // converted operands the stage completes only once they follow
+                    pre_n = min(R.s1 - s, NS);
                     for (int i = 0; i < pre_n; ++i, ++s, ++stage) {
                         const int slot = ps;
                         if (wrapped && !dk_warp_wait(&empty[slot], pph ^ 1u)) {
@@ -975,26 +1030,33 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
                             wrapped = true;
                         }
                         if (lane == 0) {
-                            mbar_arrive_expect_tx(&wfull[slot], kDkWBytes);
+                            if (pre)
+                                dk_expect_tx(&wfull[slot], kDkWBytes);
+                            else
+                                mbar_arrive_expect_tx(&wfull[slot], kDkWBytes);
                             issue_w(slot, s);
                         }
                         __syncwarp();
                     }
                     if (!ok) break;
                 }
-                if (!wait_inputs()) {
+                const bool in_ok = wait_inputs();
+                if (pre && lane == 0) {
+                    for (int i = 0; i < pre_n; ++i) {
+                        const int slot = (ps_pre + i) % NS;
+                        mbar_arrive_expect_tx(&wfull[slot], in_ok ? extra(s_pre + i) : 0u);
+                        if (in_ok) issue_x(slot, s_pre + i);
+                    }
+                }
+                __syncwarp();
+                if (!in_ok) {
                     ok = false;
                     break;
                 }
-                if (lane == 0 && R.deps != 0) {
-                    __threadfence_block();
-                    iready[q] = item;  // the stagers may convert this item's X
-                }
-                __syncwarp();
             }
             // fetched now, used after this item's stages are issued
             DkItemRec NR{};
-            if (next < a.total_items) NR = dk_load_rec<DkItemRec, 6>(a.items, next);
+            if (next < a.total_items) NR = dk_load_rec<DkItemRec, 7>(a.items, next);
             int nx2 = 0;
             if (lane == 0 && next < a.total_items)
                 nx2 = 2 * G + (int)atomicAdd(&a.ctr[kDkCtrItems], 1u);
@@ -1043,6 +1105,17 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             const int M = e.M, K = e.K;
             const int eq = (qi - 1) % kDkQueue;  // the entry's queue slot
             bool inputs = !e.chained;            // X of a dependent item: after iready
+            if (e.coop) {
+                // the layer's X is converted once: claim its units (stage, token)
+                // one at a time until none is left; the producer waits for all of
+                // them before it copies the item's operands in
+                if (e.chained && !dk_wait_ready(&iready[eq], e.item)) {
+                    ok = false;
+                    break;
+                }
+                dk_coop_convert<FMT>(a.items + e.item, e.X, e.ldx, M, K, kGlu && e.swiglu,
+                                     &a.claim[e.layer], &a.ready[e.layer], lane);
+            }
             for (int s = e.s0; s < e.s1; ++s) {
                 const int slot = ss;
                 const uint32_t ph = sph;
@@ -1768,7 +1841,7 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             __threadfence();
             a.ctr[kDkCtrItems] = 0u;
             a.ctr[kDkCtrUnitsDone] = 0u;
-            for (int l = 0; l < a.count; ++l) a.ready[l] = a.lfinal[l] = 0u;
+            for (int l = 0; l < a.count; ++l) a.ready[l] = a.lfinal[l] = a.claim[l] = 0u;
             a.ctr[kDkCtrDone] = 0u;
         }
     }
@@ -1898,6 +1971,8 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
         if (h.reads_earlier) {
             if (sc.chained == 0) sc.chained = 1;
             if (h.swiglu) sc.chained = 2;
+            if (h.M > kDkImmaMaxM)  // kDkItemCoop: converted once, during the launch
+                sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(fmt, h.M));
         } else if (src[l] == l) {
             sc.total_units += stages * h.M;
             sc.staged += (int64_t)stages * (kDkMetaBytes + dk_stage_b(fmt, h.M));
@@ -1917,8 +1992,12 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
         const int parts = dk_parts(stages, target_of(h));
         const int tiles = (h.N + kDkRows - 1) / kDkRows;
         const int bstride = kDkMetaBytes + (int)dk_stage_b(fmt, h.M);
-        const bool converts = !h.reads_earlier && src[l] == l;
-        uint8_t *B = h.reads_earlier ? nullptr : (converts ? ws + wl.staged + staged : Bs[src[l]]);
+        // A dependent layer for the fp16 engine converts its X once, during the
+        // launch (kDkItemCoop); one for the integer engine converts per item on
+        // chip (one or two tokens per stage: cheaper than a round trip)
+        const bool coop = h.reads_earlier && h.M > kDkImmaMaxM;
+        const bool converts = (!h.reads_earlier && src[l] == l) || coop;
+        uint8_t *B = h.reads_earlier && !coop ? nullptr : (converts ? ws + wl.staged + staged : Bs[src[l]]);
         Bs[l] = B;
         for (int t = 0; t < tiles; ++t)
             for (int q = 0; q < parts; ++q) {
@@ -1941,11 +2020,12 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
                 r.parts = parts;
                 r.tile_begin = tile_begin;
                 r.deps = deps[l];
-                r.need = h.reads_earlier ? (h.swiglu ? 1 : 0) : stages * h.M;
+                r.need = B ? stages * h.M : 0;
                 r.bstride = bstride;
+                r.flags = (h.swiglu ? kDkItemSwiglu : 0) | (coop ? kDkItemCoop : 0);
                 items->push_back(r);
             }
-        if (converts)
+        if (converts && !coop)
             for (int s = 0; s < stages; ++s)
                 for (int m = 0; m < h.M; ++m) {
                     DkUnitRec u{};
@@ -2034,6 +2114,7 @@ inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int
     a.ready = reinterpret_cast<uint32_t *>(b + wl.ready);
     a.lfinal = a.ready + count;
     a.ltiles = a.ready + 2 * count;
+    a.claim = a.ready + 3 * count;
     a.tile_ctr = reinterpret_cast<uint32_t *>(b + wl.tiles);
     a.partials = reinterpret_cast<int64_t *>(b + wl.partials);
     a.count = count;

@@ -131,12 +131,14 @@ def _up(v):
 
 def _ws_expected(layers, fmt=2):
     """Batch workspace, region by region (each rounded up to 256 bytes):
-    counters, one 128-byte tensor map per layer, a 96-byte record per work item
+    counters, one 128-byte tensor map per layer, a 112-byte record per work item
     (256-row tile x K-part of 2..16 stages of 128 packed bytes per row: 512
     trits at 2 bits, 640 at 1.6 bits), a 48-byte record per conversion unit
     (stage x token of a layer that reads no earlier output), a u32 per tile,
-    three u32 per layer (ready units, final tiles, tiles), 8-byte partials of
-    split tiles, and the converted activations (per stage 64 bytes plus one
+    four u32 per layer (ready units, final tiles, tiles, claimed units),
+    8-byte partials of split tiles, and the converted activations of layers
+    that read no earlier output and of dependent layers with M > 2, which
+    convert once during the launch (per stage 64 bytes plus one
     byte per trit and column of 8 per token (M = 1, 2) or two bytes per trit
     and token rounded up to even (M >= 3)).  A layer with a dependency has its
     items sized to spread it over about 148 CTAs (at most 8 parts per tile, 2
@@ -166,15 +168,17 @@ def _ws_expected(layers, fmt=2):
         items += t * parts
         tiles += t
         key = (d.get("dX", A), d.get("ldx", d["K"] + (-d["K"]) % 8), d["K"], d["M"])
+        b = 8 * 128 * g * d["M"] if d["M"] <= 2 else 2 * 128 * g * (d["M"] + d["M"] % 2)
         if not d.get("flags", 0) and key not in seen:
             seen.add(key)
             units += stages * d["M"]
-            b = 8 * 128 * g * d["M"] if d["M"] <= 2 else 2 * 128 * g * (d["M"] + d["M"] % 2)
+            staged += stages * (64 + b)
+        elif d.get("flags", 0) and d["M"] > 2:
             staged += stages * (64 + b)
         if parts > 1:
             slots += t * parts * 256 * d["M"]
     off = 256
-    for size in (128 * len(layers), 96 * items, 48 * units, 12 * len(layers), 4 * tiles, 8 * slots,
+    for size in (128 * len(layers), 112 * items, 48 * units, 16 * len(layers), 4 * tiles, 8 * slots,
                  staged):
         off = _up(off + size)
     return off
