@@ -1,5 +1,5 @@
-// tl_decode.cuh -- a batch of decode-shaped 2-bit ternary layers (M = 1..8
-// tokens each) in ONE persistent launch:
+// tl_decode.cuh -- a batch of decode-shaped ternary layers (M = 1..8 tokens
+// each; 2-bit or 1.6-bit packing) in ONE persistent launch:
 //   for every layer l:  Y_l[m][n] = fp16_rn(alpha_l * sum_k T_l[n][k] X_l[m][k]).
 //
 // Decoding streams every packed weight once and is bound by memory bandwidth
@@ -26,21 +26,29 @@
 //    halves d * 2^(2j-24) (one AND per register); one accumulator per digit
 //    position, combined with exact power-of-two scales; sum_k x_k is
 //    subtracted at the end (d = t + 1).
+//  * Base 3 (1.6-bit, decode2_kernel<16>): the same roles and engines, with
+//    the digits' quotients floor(v / 3^p) taken two bytes per IMAD in 16-bit
+//    lanes (see "base 3" below): the integer engine multiplies the quotients
+//    themselves against telescoped activations, the fp16 engine the digits.
 //
-// Weights arrive by TMA in boxes of 256 rows x 128 bytes (512 trits per row)
-// with the 128-byte swizzle, one box per stage.  A consumer lane (g, c) reads
-// 16-byte chunk 4v + c of rows g and g + 8 of a 16-row tile; MMA row g is physical row pi(g) = ((g & 1) << 2) | (g >> 1), so
-// the two rows of every quarter-warp differ in bit 2 and each LDS.128 touches
-// every bank once.
+// Weights arrive by TMA in boxes of 256 rows x 128 bytes (512 trits per row
+// at 2 bits, 640 at 1.6 bits) with the 128-byte swizzle, one box per stage.
+// A consumer lane (g, c) reads 16-byte chunk 4v + c of rows g and g + 8 of a
+// 16-row tile; MMA row g is physical row pi(g) = ((g & 1) << 2) | (g >> 1),
+// so the two rows of every quarter-warp differ in bit 2 and each LDS.128
+// touches every bank once.
 //
 // Activations go into the B layout of their engine once per (layer, stage),
 // not once per item: every warp except the producer first converts such
 // units (unit u by converting warp u mod their number) into the workspace
 // and counts them per layer; a stage's converted operands then arrive by one
-// bulk copy next to its weights.  Layers flagged as reading an earlier
-// layer's output (their X is written during this launch), and the first item
-// of every CTA (so no CTA starts by waiting for others), are converted per
-// item instead, from X in global memory, by stager warps.
+// bulk copy next to its weights.  The first item of every CTA (so no CTA
+// starts by waiting for others) and items of layers flagged as reading an
+// earlier layer's output (their X is written during this launch) for the
+// integer engine are converted per item instead, from X in global memory, by
+// stager warps; such layers for the fp16 engine convert their X once, after
+// the layers they read are complete, by the stagers of their items.  A
+// dependent layer waits only for the earlier layers whose Y overlaps its X.
 //
 // Warp roles of a CTA (768 threads):
 //  * warp 0, producer: issues each stage's copies into a ring and queues items
@@ -1320,511 +1328,511 @@ __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_con
             const int b = pi % NB;
             uint8_t *pb = parts + b * lay.parts;
             if constexpr (FMT == 2) {
-            if (M == 1) {
-                // ---- integer engine, one token: one accumulator per digit
-                // position j (A = digits * 4^j, one AND per register) ----
-                int acc[2][4][4];  // [tile][digit position][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[t][j][0] = acc[t][j][1] = acc[t][j][2] = acc[t][j][3] = 0;
-                int64_t qsum = 0;
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
+                if (M == 1) {
+                    // ---- integer engine, one token: one accumulator per digit
+                    // position j (A = digits * 4^j, one AND per register) ----
+                    int acc[2][4][4];  // [tile][digit position][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[t][j][0] = acc[t][j][1] = acc[t][j][2] = acc[t][j][3] = 0;
+                    int64_t qsum = 0;
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A00 = dk_lds128(wb);                     // tile 2tp, row g
+                        const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);   // tile 2tp, row g + 8
+                        const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);  // tile 2tp + 1, row g
+                        const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);  // tile 2tp + 1, row g + 8
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        qsum += reinterpret_cast<const int64_t *>(sb)[0];
+                        const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
+    #pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {
+                            const int i0 = 2 * pr, i1 = i0 + 1;
+                            const uint4 B0 = dk_lds128(xg + i0 * 512), B1 = dk_lds128(xg + i1 * 512);
+    #pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint32_t m = 0x03030303u << (2 * j);
+                                const uint32_t b0 = dk_word(B0, j), b1 = dk_word(B1, j);
+                                mma_u8_16832(acc[0][j], dk_word(A00, i0) & m, dk_word(A01, i0) & m,
+                                             dk_word(A00, i1) & m, dk_word(A01, i1) & m, b0, b1);
+                                mma_u8_16832(acc[1][j], dk_word(A10, i0) & m, dk_word(A11, i0) & m,
+                                             dk_word(A10, i1) & m, dk_word(A11, i1) & m, b0, b1);
+                            }
+                        }
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
                         break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A00 = dk_lds128(wb);                     // tile 2tp, row g
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);   // tile 2tp, row g + 8
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);  // tile 2tp + 1, row g
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);  // tile 2tp + 1, row g + 8
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    qsum += reinterpret_cast<const int64_t *>(sb)[0];
-                    const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
-#pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        const int i0 = 2 * pr, i1 = i0 + 1;
-                        const uint4 B0 = dk_lds128(xg + i0 * 512), B1 = dk_lds128(xg + i1 * 512);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t m = 0x03030303u << (2 * j);
-                            const uint32_t b0 = dk_word(B0, j), b1 = dk_word(B1, j);
-                            mma_u8_16832(acc[0][j], dk_word(A00, i0) & m, dk_word(A01, i0) & m,
-                                         dk_word(A00, i1) & m, dk_word(A01, i1) & m, b0, b1);
-                            mma_u8_16832(acc[1][j], dk_word(A10, i0) & m, dk_word(A11, i0) & m,
-                                         dk_word(A10, i1) & m, dk_word(A11, i1) & m, b0, b1);
+                    // V = sum_p 256^p S_p - 2^40 S_ones - Q; this lane holds columns
+                    // 2c, 2c + 1 (planes 2c, 2c + 1, or the ones column at c = 3)
+                    // D = 64 S exactly: position j carries 4^j, so acc0*64 + acc1*16 +
+                    // acc2*4 + acc3 = 64 sum_j acc_j 4^-j (below 2^31 for items of at most
+                    // kDkMaxItemStages stages); lane c's columns give t_c = D_2c + 256 D_2c+1
+                    // (lane 3: the ones column), and lane 0 forms
+                    // 64 V = t_0 + 2^16 t_1 + 2^32 t_2 - 2^40 t_3 - 64 Q (modulo 2^64).
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+    #pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            uint32_t d[2];
+    #pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int q = 2 * rr + u;
+                                d[u] = (uint32_t)(acc[t][0][q] * 64 + acc[t][1][q] * 16 + acc[t][2][q] * 4 +
+                                                  acc[t][3][q]);
+                            }
+                            const uint64_t tc = c < 3 ? (uint64_t)d[0] + ((uint64_t)d[1] << 8) : (uint64_t)d[0];
+                            const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
+                            const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
+                            const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
+                            if (c == 0) {
+                                uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 40);
+                                if (qv == 0) v64 -= (uint64_t)qsum << 6;
+                                reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] =
+                                    (int64_t)v64 >> 6;
+                            }
                         }
                     }
-                    release(slot);
-                }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                // V = sum_p 256^p S_p - 2^40 S_ones - Q; this lane holds columns
-                // 2c, 2c + 1 (planes 2c, 2c + 1, or the ones column at c = 3)
-                // D = 64 S exactly: position j carries 4^j, so acc0*64 + acc1*16 +
-                // acc2*4 + acc3 = 64 sum_j acc_j 4^-j (below 2^31 for items of at most
-                // kDkMaxItemStages stages); lane c's columns give t_c = D_2c + 256 D_2c+1
-                // (lane 3: the ones column), and lane 0 forms
-                // 64 V = t_0 + 2^16 t_1 + 2^32 t_2 - 2^40 t_3 - 64 Q (modulo 2^64).
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        uint32_t d[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int q = 2 * rr + u;
-                            d[u] = (uint32_t)(acc[t][0][q] * 64 + acc[t][1][q] * 16 + acc[t][2][q] * 4 +
-                                              acc[t][3][q]);
+                } else if (M == 2) {
+                    // ---- integer engine, two tokens: two column groups share the
+                    // decoded digits (shifted to the low bits, one accumulator) ----
+                    int iacc[2][2][4];  // [tile][column group][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                        for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
+                    int64_t qsum0 = 0, qsum1 = 0;
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
                         }
-                        const uint64_t tc = c < 3 ? (uint64_t)d[0] + ((uint64_t)d[1] << 8) : (uint64_t)d[0];
-                        const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
-                        const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
-                        const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
-                        if (c == 0) {
-                            uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 40);
-                            if (qv == 0) v64 -= (uint64_t)qsum << 6;
-                            reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] =
-                                (int64_t)v64 >> 6;
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A00 = dk_lds128(wb);
+                        const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
+                        const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
+                        const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
+                        qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
+                        const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
+    #pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {
+                            const int i0 = 2 * pr, i1 = i0 + 1;
+                            const uint4 B00 = dk_lds128(xg + i0 * 512), B01 = dk_lds128(xg + i1 * 512);
+                            const uint4 B10 = dk_lds128(xg + 4096 + i0 * 512);
+                            const uint4 B11 = dk_lds128(xg + 4096 + i1 * 512);
+    #pragma unroll 2
+                            for (int j = 0; j < 4; ++j) {
+                                constexpr uint32_t m = 0x03030303u;
+                                const uint32_t a00 = (dk_word(A00, i0) >> (2 * j)) & m;
+                                const uint32_t a01 = (dk_word(A01, i0) >> (2 * j)) & m;
+                                const uint32_t a02 = (dk_word(A00, i1) >> (2 * j)) & m;
+                                const uint32_t a03 = (dk_word(A01, i1) >> (2 * j)) & m;
+                                const uint32_t a10 = (dk_word(A10, i0) >> (2 * j)) & m;
+                                const uint32_t a11 = (dk_word(A11, i0) >> (2 * j)) & m;
+                                const uint32_t a12 = (dk_word(A10, i1) >> (2 * j)) & m;
+                                const uint32_t a13 = (dk_word(A11, i1) >> (2 * j)) & m;
+                                const uint32_t b00 = dk_word(B00, j), b01 = dk_word(B01, j);
+                                const uint32_t b10 = dk_word(B10, j), b11 = dk_word(B11, j);
+                                mma_u8_16832(iacc[0][0], a00, a01, a02, a03, b00, b01);
+                                mma_u8_16832(iacc[1][0], a10, a11, a12, a13, b00, b01);
+                                mma_u8_16832(iacc[0][1], a00, a01, a02, a03, b10, b11);
+                                mma_u8_16832(iacc[1][1], a10, a11, a12, a13, b10, b11);
+                            }
                         }
+                        release(slot);
                     }
-                }
-            } else if (M == 2) {
-                // ---- integer engine, two tokens: two column groups share the
-                // decoded digits (shifted to the low bits, one accumulator) ----
-                int iacc[2][2][4];  // [tile][column group][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
-                int64_t qsum0 = 0, qsum1 = 0;
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
                         break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A00 = dk_lds128(wb);
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
-                    qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
-                    const uint8_t *xg = sb + kDkMetaBytes + ((v * 32 + g) * 4 + c) * 16;
-#pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        const int i0 = 2 * pr, i1 = i0 + 1;
-                        const uint4 B00 = dk_lds128(xg + i0 * 512), B01 = dk_lds128(xg + i1 * 512);
-                        const uint4 B10 = dk_lds128(xg + 4096 + i0 * 512);
-                        const uint4 B11 = dk_lds128(xg + 4096 + i1 * 512);
-#pragma unroll 2
-                        for (int j = 0; j < 4; ++j) {
-                            constexpr uint32_t m = 0x03030303u;
-                            const uint32_t a00 = (dk_word(A00, i0) >> (2 * j)) & m;
-                            const uint32_t a01 = (dk_word(A01, i0) >> (2 * j)) & m;
-                            const uint32_t a02 = (dk_word(A00, i1) >> (2 * j)) & m;
-                            const uint32_t a03 = (dk_word(A01, i1) >> (2 * j)) & m;
-                            const uint32_t a10 = (dk_word(A10, i0) >> (2 * j)) & m;
-                            const uint32_t a11 = (dk_word(A11, i0) >> (2 * j)) & m;
-                            const uint32_t a12 = (dk_word(A10, i1) >> (2 * j)) & m;
-                            const uint32_t a13 = (dk_word(A11, i1) >> (2 * j)) & m;
-                            const uint32_t b00 = dk_word(B00, j), b01 = dk_word(B01, j);
-                            const uint32_t b10 = dk_word(B10, j), b11 = dk_word(B11, j);
-                            mma_u8_16832(iacc[0][0], a00, a01, a02, a03, b00, b01);
-                            mma_u8_16832(iacc[1][0], a10, a11, a12, a13, b00, b01);
-                            mma_u8_16832(iacc[0][1], a00, a01, a02, a03, b10, b11);
-                            mma_u8_16832(iacc[1][1], a10, a11, a12, a13, b10, b11);
+                    // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
+                    // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+    #pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            const int64_t d0 = iacc[t][0][2 * rr], d1 = iacc[t][0][2 * rr + 1];
+                            const int64_t e0 = iacc[t][1][2 * rr], e1 = iacc[t][1][2 * rr + 1];
+                            int64_t v0 = 0, v1 = 0;
+                            if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
+                            else v1 = d0 + (d1 << 8);
+                            if (c < 2) {
+                                v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
+                            } else if (c == 2) {
+                                v0 -= e0 << 40;
+                                v1 -= e0 << 40;
+                            }
+                            v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                            v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+                            v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                            v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+                            if (qv == 0) {
+                                v0 -= qsum0;
+                                v1 -= qsum1;
+                            }
+                            if (c == 0) {
+                                int64_t *p = reinterpret_cast<int64_t *>(pb);
+                                p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                                p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
+                            }
                         }
                     }
-                    release(slot);
-                }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
-                // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int64_t d0 = iacc[t][0][2 * rr], d1 = iacc[t][0][2 * rr + 1];
-                        const int64_t e0 = iacc[t][1][2 * rr], e1 = iacc[t][1][2 * rr + 1];
-                        int64_t v0 = 0, v1 = 0;
-                        if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
-                        else v1 = d0 + (d1 << 8);
-                        if (c < 2) {
-                            v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
-                        } else if (c == 2) {
-                            v0 -= e0 << 40;
-                            v1 -= e0 << 40;
+                } else {
+                    // ---- fp16 engine ----
+                    const int Mp = M + (M & 1);
+                    float facc[2][4][4];  // [tile][digit position][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            facc[t][q][0] = facc[t][q][1] = facc[t][q][2] = facc[t][q][3] = 0.f;
+                    float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
                         }
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-                        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-                        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A00 = dk_lds128(wb);
+                        const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
+                        const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
+                        const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        const float *mt = reinterpret_cast<const float *>(sb);
+                        if (2 * c < M) sx0 += mt[2 * c];
+                        if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
+                        const uint8_t *xb = sb + kDkMetaBytes;
+    #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint4 B0 = make_uint4(0u, 0u, 0u, 0u), B1 = B0;
+                            if (g < M) {
+                                const int w = (4 * v + c) * 4 + i;
+                                B0 = dk_lds128(xb + dk_hblock(w, g, 0, Mp));
+                                B1 = dk_lds128(xb + dk_hblock(w, g, 1, Mp));
+                            }
+                            const uint32_t bb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
+                            const uint32_t W0 = dk_word(A00, i), V0 = dk_word(A01, i);
+                            const uint32_t W1 = dk_word(A10, i), V1 = dk_word(A11, i);
+                            const uint32_t hW0 = W0 >> 8, hV0 = V0 >> 8, hW1 = W1 >> 8, hV1 = V1 >> 8;
+    #pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint32_t m = 0x00030003u << (2 * j);
+                                mma_16816(facc[0][j], W0 & m, V0 & m, hW0 & m, hV0 & m, bb[2 * j],
+                                          bb[2 * j + 1]);
+                                mma_16816(facc[1][j], W1 & m, V1 & m, hW1 & m, hV1 & m, bb[2 * j],
+                                          bb[2 * j + 1]);
+                            }
+                        }
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                        break;
+                    float *p = reinterpret_cast<float *>(pb);
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        float sv[4];
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            sv[q] = facc[t][0][q] * 16777216.0f + facc[t][1][q] * 4194304.0f +
+                                    facc[t][2][q] * 1048576.0f + facc[t][3][q] * 262144.0f;
                         if (qv == 0) {
-                            v0 -= qsum0;
-                            v1 -= qsum1;
+                            sv[0] -= sx0;
+                            sv[1] -= sx1;
+                            sv[2] -= sx0;
+                            sv[3] -= sx1;
                         }
-                        if (c == 0) {
-                            int64_t *p = reinterpret_cast<int64_t *>(pb);
-                            p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
-                            p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
+                        const int m0 = 2 * c, m1 = 2 * c + 1;
+                        if (m0 < M) {
+                            p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
+                            p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
+                        }
+                        if (m1 < M) {
+                            p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
+                            p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
                         }
                     }
                 }
             } else {
-                // ---- fp16 engine ----
-                const int Mp = M + (M & 1);
-                float facc[2][4][4];  // [tile][digit position][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        facc[t][q][0] = facc[t][q][1] = facc[t][q][2] = facc[t][q][3] = 0.f;
-                float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A00 = dk_lds128(wb);
-                    const uint4 A01 = dk_lds128(wb + 8 * kDkStageW);
-                    const uint4 A10 = dk_lds128(wb + 16 * kDkStageW);
-                    const uint4 A11 = dk_lds128(wb + 24 * kDkStageW);
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    const float *mt = reinterpret_cast<const float *>(sb);
-                    if (2 * c < M) sx0 += mt[2 * c];
-                    if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
-                    const uint8_t *xb = sb + kDkMetaBytes;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4 B0 = make_uint4(0u, 0u, 0u, 0u), B1 = B0;
-                        if (g < M) {
-                            const int w = (4 * v + c) * 4 + i;
-                            B0 = dk_lds128(xb + dk_hblock(w, g, 0, Mp));
-                            B1 = dk_lds128(xb + dk_hblock(w, g, 1, Mp));
+                if (M == 1) {
+                    // ---- base-3 integer engine, one token: positions p = 0..4 (the
+                    // bytes, then their quotients by 3, 9, 27, 81) share one
+                    // accumulator; B carries each position's activations ----
+                    int acc[2][4];  // [tile][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0;
+                    int64_t qsum = 0;
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
                         }
-                        const uint32_t bb[8] = {B0.x, B0.y, B0.z, B0.w, B1.x, B1.y, B1.z, B1.w};
-                        const uint32_t W0 = dk_word(A00, i), V0 = dk_word(A01, i);
-                        const uint32_t W1 = dk_word(A10, i), V1 = dk_word(A11, i);
-                        const uint32_t hW0 = W0 >> 8, hV0 = V0 >> 8, hW1 = W1 >> 8, hV1 = V1 >> 8;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t m = 0x00030003u << (2 * j);
-                            mma_16816(facc[0][j], W0 & m, V0 & m, hW0 & m, hV0 & m, bb[2 * j],
-                                      bb[2 * j + 1]);
-                            mma_16816(facc[1][j], W1 & m, V1 & m, hW1 & m, hV1 & m, bb[2 * j],
-                                      bb[2 * j + 1]);
-                        }
-                    }
-                    release(slot);
-                }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                float *p = reinterpret_cast<float *>(pb);
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    float sv[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        sv[q] = facc[t][0][q] * 16777216.0f + facc[t][1][q] * 4194304.0f +
-                                facc[t][2][q] * 1048576.0f + facc[t][3][q] * 262144.0f;
-                    if (qv == 0) {
-                        sv[0] -= sx0;
-                        sv[1] -= sx1;
-                        sv[2] -= sx0;
-                        sv[3] -= sx1;
-                    }
-                    const int m0 = 2 * c, m1 = 2 * c + 1;
-                    if (m0 < M) {
-                        p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
-                        p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
-                    }
-                    if (m1 < M) {
-                        p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
-                        p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
-                    }
-                }
-            }
-            } else {
-            if (M == 1) {
-                // ---- base-3 integer engine, one token: positions p = 0..4 (the
-                // bytes, then their quotients by 3, 9, 27, 81) share one
-                // accumulator; B carries each position's activations ----
-                int acc[2][4];  // [tile][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0;
-                int64_t qsum = 0;
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
-                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    qsum += reinterpret_cast<const int64_t *>(sb)[0];
-                    const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
-#pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        // [tile][row g / g + 8][word 2pr / 2pr + 1]: A words, and their
-                        // even / odd bytes in 16-bit lanes
-                        uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
-#pragma unroll
-                        for (int t = 0; t < 2; ++t)
-#pragma unroll
-                            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
-                                    E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
-                                    O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
-                                }
-#pragma unroll
-                        for (int p = 0; p < 5; ++p) {
-                            if (p > 0) {
-#pragma unroll
-                                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                                    for (int r = 0; r < 2; ++r)
-#pragma unroll
-                                        for (int h = 0; h < 2; ++h) {
-                                            const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
-                                            const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
-                                            P[t][r][h] = prmt(tE, tO, 0x7351u);
-                                            E[t][r][h] = prmt(tE, 0u, 0x4341u);
-                                            O[t][r][h] = prmt(tO, 0u, 0x4341u);
-                                        }
-                            }
-                            const uint2 bq = *reinterpret_cast<const uint2 *>(xg + dk_i3off(0, pr, p, 0, 0));
-#pragma unroll
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                               {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        qsum += reinterpret_cast<const int64_t *>(sb)[0];
+                        const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
+    #pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {
+                            // [tile][row g / g + 8][word 2pr / 2pr + 1]: A words, and their
+                            // even / odd bytes in 16-bit lanes
+                            uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
+    #pragma unroll
                             for (int t = 0; t < 2; ++t)
-                                mma_u8_16832(acc[t], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1], bq.x,
-                                             bq.y);
-                        }
-                    }
-                    release(slot);
-                }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                // V = sum_p 256^p S_p - 2^42 S_ones - Q; lane c holds columns 2c,
-                // 2c + 1 (planes, or the ones column at c = 3), and lane 0 of the
-                // quad forms V (modulo 2^64)
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const uint64_t d0 = (uint32_t)acc[t][2 * rr], d1 = (uint32_t)acc[t][2 * rr + 1];
-                        const uint64_t tc = c < 3 ? d0 + (d1 << 8) : d0;
-                        const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
-                        const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
-                        const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
-                        if (c == 0) {
-                            uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 42);
-                            if (qv == 0) v64 -= (uint64_t)qsum;
-                            reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] = (int64_t)v64;
-                        }
-                    }
-                }
-            } else if (M == 2) {
-                // ---- base-3 integer engine, two tokens: two column groups ----
-                int iacc[2][2][4];  // [tile][column group][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
-                int64_t qsum0 = 0, qsum1 = 0;
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
-                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
-                    qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
-                    const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
-#pragma unroll
-                    for (int pr = 0; pr < 2; ++pr) {
-                        uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
-#pragma unroll
-                        for (int t = 0; t < 2; ++t)
-#pragma unroll
-                            for (int r = 0; r < 2; ++r)
-#pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
-                                    E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
-                                    O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
-                                }
-#pragma unroll
-                        for (int p = 0; p < 5; ++p) {
-                            if (p > 0) {
-#pragma unroll
-                                for (int t = 0; t < 2; ++t)
-#pragma unroll
-                                    for (int r = 0; r < 2; ++r)
-#pragma unroll
-                                        for (int h = 0; h < 2; ++h) {
-                                            const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
-                                            const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
-                                            P[t][r][h] = prmt(tE, tO, 0x7351u);
-                                            E[t][r][h] = prmt(tE, 0u, 0x4341u);
-                                            O[t][r][h] = prmt(tO, 0u, 0x4341u);
-                                        }
-                            }
-                            const uint32_t off = dk_i3off(0, pr, p, 0, 0);
-                            const uint2 bq0 = *reinterpret_cast<const uint2 *>(xg + off);
-                            const uint2 bq1 = *reinterpret_cast<const uint2 *>(xg + 5 * 1024 + off);
-#pragma unroll
-                            for (int t = 0; t < 2; ++t) {
-                                mma_u8_16832(iacc[t][0], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
-                                             bq0.x, bq0.y);
-                                mma_u8_16832(iacc[t][1], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
-                                             bq1.x, bq1.y);
-                            }
-                        }
-                    }
-                    release(slot);
-                }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
-                // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-#pragma unroll
-                    for (int rr = 0; rr < 2; ++rr) {
-                        const int64_t d0 = (uint32_t)iacc[t][0][2 * rr], d1 = (uint32_t)iacc[t][0][2 * rr + 1];
-                        const int64_t e0 = (uint32_t)iacc[t][1][2 * rr], e1 = (uint32_t)iacc[t][1][2 * rr + 1];
-                        int64_t v0 = 0, v1 = 0;
-                        if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
-                        else v1 = d0 + (d1 << 8);
-                        if (c < 2) {
-                            v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
-                        } else if (c == 2) {
-                            v0 -= e0 << 42;
-                            v1 -= e0 << 42;
-                        }
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
-                        v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
-                        v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
-                        v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
-                        if (qv == 0) {
-                            v0 -= qsum0;
-                            v1 -= qsum1;
-                        }
-                        if (c == 0) {
-                            int64_t *p = reinterpret_cast<int64_t *>(pb);
-                            p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
-                            p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
-                        }
-                    }
-                }
-            } else {
-                // ---- base-3 fp16 engine: digits as subnormal halves d 2^-24 in
-                // 16-bit lanes (even bytes, odd bytes), one accumulator ----
-                const int Mp = M + (M & 1);
-                float facc[2][4];  // [tile][D]
-#pragma unroll
-                for (int t = 0; t < 2; ++t) facc[t][0] = facc[t][1] = facc[t][2] = facc[t][3] = 0.f;
-                float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
-                for (int s = e.s0; s < e.s1; ++s) {
-                    const int slot = cs;
-                    if (!wait_stage(slot)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint8_t *wb = wring + slot * kDkWBytes + aoff;
-                    const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
-                                           {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
-                    const uint8_t *sb = sslot + slot * lay.slot_b;
-                    const float *mt = reinterpret_cast<const float *>(sb);
-                    if (2 * c < M) sx0 += mt[2 * c];
-                    if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
-                    const uint8_t *xb = sb + kDkMetaBytes;
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint32_t E[2][2], O[2][2];  // [tile][row g / g + 8]
-#pragma unroll
-                        for (int t = 0; t < 2; ++t)
-#pragma unroll
-                            for (int r = 0; r < 2; ++r) {
-                                const uint32_t W = dk_word(A[t][r], i);
-                                E[t][r] = prmt(W, 0u, 0x4240u);
-                                O[t][r] = prmt(W, 0u, 0x4341u);
-                            }
-#pragma unroll
-                        for (int p = 0; p < 5; ++p) {
-                            uint2 bq = make_uint2(0u, 0u);
-                            if (g < M) bq = *reinterpret_cast<const uint2 *>(xb + dk_h3off(v, i, p, g, c, Mp));
-                            uint32_t dE[2][2], dO[2][2];
-#pragma unroll
-                            for (int t = 0; t < 2; ++t)
-#pragma unroll
-                                for (int r = 0; r < 2; ++r) {
-                                    if (p < 4) {
-                                        // d_p = q_p - 3 q_{p+1} per lane (never negative)
-                                        const uint32_t e1 = prmt(E[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
-                                        const uint32_t o1 = prmt(O[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
-                                        dE[t][r] = E[t][r] - 3u * e1;
-                                        dO[t][r] = O[t][r] - 3u * o1;
-                                        E[t][r] = e1;
-                                        O[t][r] = o1;
-                                    } else {
-                                        dE[t][r] = E[t][r];
-                                        dO[t][r] = O[t][r];
+    #pragma unroll
+                                for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
+                                        E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
+                                        O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
                                     }
+    #pragma unroll
+                            for (int p = 0; p < 5; ++p) {
+                                if (p > 0) {
+    #pragma unroll
+                                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                                        for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                                            for (int h = 0; h < 2; ++h) {
+                                                const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
+                                                const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
+                                                P[t][r][h] = prmt(tE, tO, 0x7351u);
+                                                E[t][r][h] = prmt(tE, 0u, 0x4341u);
+                                                O[t][r][h] = prmt(tO, 0u, 0x4341u);
+                                            }
                                 }
-#pragma unroll
-                            for (int t = 0; t < 2; ++t)
-                                mma_16816(facc[t], dE[t][0], dE[t][1], dO[t][0], dO[t][1], bq.x, bq.y);
+                                const uint2 bq = *reinterpret_cast<const uint2 *>(xg + dk_i3off(0, pr, p, 0, 0));
+    #pragma unroll
+                                for (int t = 0; t < 2; ++t)
+                                    mma_u8_16832(acc[t], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1], bq.x,
+                                                 bq.y);
+                            }
+                        }
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                        break;
+                    // V = sum_p 256^p S_p - 2^42 S_ones - Q; lane c holds columns 2c,
+                    // 2c + 1 (planes, or the ones column at c = 3), and lane 0 of the
+                    // quad forms V (modulo 2^64)
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+    #pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            const uint64_t d0 = (uint32_t)acc[t][2 * rr], d1 = (uint32_t)acc[t][2 * rr + 1];
+                            const uint64_t tc = c < 3 ? d0 + (d1 << 8) : d0;
+                            const uint64_t t1 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 1);
+                            const uint64_t t2 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 2);
+                            const uint64_t t3 = __shfl_sync(0xffffffffu, tc, (lane & ~3) | 3);
+                            if (c == 0) {
+                                uint64_t v64 = tc + (t1 << 16) + (t2 << 32) - (t3 << 42);
+                                if (qv == 0) v64 -= (uint64_t)qsum;
+                                reinterpret_cast<int64_t *>(pb)[(cw * 2 + t) * 16 + g + 8 * rr] = (int64_t)v64;
+                            }
                         }
                     }
-                    release(slot);
+                } else if (M == 2) {
+                    // ---- base-3 integer engine, two tokens: two column groups ----
+                    int iacc[2][2][4];  // [tile][column group][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                        for (int q = 0; q < 8; ++q) iacc[t][q >> 2][q & 3] = 0;
+                    int64_t qsum0 = 0, qsum1 = 0;
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                               {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        qsum0 += reinterpret_cast<const int64_t *>(sb)[0];
+                        qsum1 += reinterpret_cast<const int64_t *>(sb)[1];
+                        const uint8_t *xg = sb + kDkMetaBytes + dk_i3off(v, 0, 0, g, c);
+    #pragma unroll
+                        for (int pr = 0; pr < 2; ++pr) {
+                            uint32_t P[2][2][2], E[2][2][2], O[2][2][2];
+    #pragma unroll
+                            for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                                for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                                    for (int h = 0; h < 2; ++h) {
+                                        P[t][r][h] = dk_word(A[t][r], 2 * pr + h);
+                                        E[t][r][h] = prmt(P[t][r][h], 0u, 0x4240u);
+                                        O[t][r][h] = prmt(P[t][r][h], 0u, 0x4341u);
+                                    }
+    #pragma unroll
+                            for (int p = 0; p < 5; ++p) {
+                                if (p > 0) {
+    #pragma unroll
+                                    for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                                        for (int r = 0; r < 2; ++r)
+    #pragma unroll
+                                            for (int h = 0; h < 2; ++h) {
+                                                const uint32_t tE = E[t][r][h] * 85u + 0x00550055u;
+                                                const uint32_t tO = O[t][r][h] * 85u + 0x00550055u;
+                                                P[t][r][h] = prmt(tE, tO, 0x7351u);
+                                                E[t][r][h] = prmt(tE, 0u, 0x4341u);
+                                                O[t][r][h] = prmt(tO, 0u, 0x4341u);
+                                            }
+                                }
+                                const uint32_t off = dk_i3off(0, pr, p, 0, 0);
+                                const uint2 bq0 = *reinterpret_cast<const uint2 *>(xg + off);
+                                const uint2 bq1 = *reinterpret_cast<const uint2 *>(xg + 5 * 1024 + off);
+    #pragma unroll
+                                for (int t = 0; t < 2; ++t) {
+                                    mma_u8_16832(iacc[t][0], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
+                                                 bq0.x, bq0.y);
+                                    mma_u8_16832(iacc[t][1], P[t][0][0], P[t][1][0], P[t][0][1], P[t][1][1],
+                                                 bq1.x, bq1.y);
+                                }
+                            }
+                        }
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                        break;
+                    // columns: token 0 planes 0..5 (group 0, c 0..2), token 1 planes
+                    // 0..1 (group 0, c 3) and 2..5 (group 1, c 0..1), ones (group 1, c 2)
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+    #pragma unroll
+                        for (int rr = 0; rr < 2; ++rr) {
+                            const int64_t d0 = (uint32_t)iacc[t][0][2 * rr], d1 = (uint32_t)iacc[t][0][2 * rr + 1];
+                            const int64_t e0 = (uint32_t)iacc[t][1][2 * rr], e1 = (uint32_t)iacc[t][1][2 * rr + 1];
+                            int64_t v0 = 0, v1 = 0;
+                            if (c < 3) v0 = (d0 << (16 * c)) + (d1 << (16 * c + 8));
+                            else v1 = d0 + (d1 << 8);
+                            if (c < 2) {
+                                v1 += (e0 << (16 * c + 16)) + (e1 << (16 * c + 24));
+                            } else if (c == 2) {
+                                v0 -= e0 << 42;
+                                v1 -= e0 << 42;
+                            }
+                            v0 += __shfl_xor_sync(0xffffffffu, v0, 1);
+                            v0 += __shfl_xor_sync(0xffffffffu, v0, 2);
+                            v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+                            v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
+                            if (qv == 0) {
+                                v0 -= qsum0;
+                                v1 -= qsum1;
+                            }
+                            if (c == 0) {
+                                int64_t *p = reinterpret_cast<int64_t *>(pb);
+                                p[(cw * 2 + t) * 16 + g + 8 * rr] = v0;
+                                p[((16 + cw) * 2 + t) * 16 + g + 8 * rr] = v1;
+                            }
+                        }
+                    }
+                } else {
+                    // ---- base-3 fp16 engine: digits as subnormal halves d 2^-24 in
+                    // 16-bit lanes (even bytes, odd bytes), one accumulator ----
+                    const int Mp = M + (M & 1);
+                    float facc[2][4];  // [tile][D]
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) facc[t][0] = facc[t][1] = facc[t][2] = facc[t][3] = 0.f;
+                    float sx0 = 0.f, sx1 = 0.f;  // sum x of this lane's tokens 2c, 2c + 1
+                    for (int s = e.s0; s < e.s1; ++s) {
+                        const int slot = cs;
+                        if (!wait_stage(slot)) {
+                            ok = false;
+                            break;
+                        }
+                        const uint8_t *wb = wring + slot * kDkWBytes + aoff;
+                        const uint4 A[2][2] = {{dk_lds128(wb), dk_lds128(wb + 8 * kDkStageW)},
+                                               {dk_lds128(wb + 16 * kDkStageW), dk_lds128(wb + 24 * kDkStageW)}};
+                        const uint8_t *sb = sslot + slot * lay.slot_b;
+                        const float *mt = reinterpret_cast<const float *>(sb);
+                        if (2 * c < M) sx0 += mt[2 * c];
+                        if (2 * c + 1 < M) sx1 += mt[2 * c + 1];
+                        const uint8_t *xb = sb + kDkMetaBytes;
+    #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t E[2][2], O[2][2];  // [tile][row g / g + 8]
+    #pragma unroll
+                            for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                                for (int r = 0; r < 2; ++r) {
+                                    const uint32_t W = dk_word(A[t][r], i);
+                                    E[t][r] = prmt(W, 0u, 0x4240u);
+                                    O[t][r] = prmt(W, 0u, 0x4341u);
+                                }
+    #pragma unroll
+                            for (int p = 0; p < 5; ++p) {
+                                uint2 bq = make_uint2(0u, 0u);
+                                if (g < M) bq = *reinterpret_cast<const uint2 *>(xb + dk_h3off(v, i, p, g, c, Mp));
+                                uint32_t dE[2][2], dO[2][2];
+    #pragma unroll
+                                for (int t = 0; t < 2; ++t)
+    #pragma unroll
+                                    for (int r = 0; r < 2; ++r) {
+                                        if (p < 4) {
+                                            // d_p = q_p - 3 q_{p+1} per lane (never negative)
+                                            const uint32_t e1 = prmt(E[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
+                                            const uint32_t o1 = prmt(O[t][r] * 85u + 0x00550055u, 0u, 0x4341u);
+                                            dE[t][r] = E[t][r] - 3u * e1;
+                                            dO[t][r] = O[t][r] - 3u * o1;
+                                            E[t][r] = e1;
+                                            O[t][r] = o1;
+                                        } else {
+                                            dE[t][r] = E[t][r];
+                                            dO[t][r] = O[t][r];
+                                        }
+                                    }
+    #pragma unroll
+                                for (int t = 0; t < 2; ++t)
+                                    mma_16816(facc[t], dE[t][0], dE[t][1], dO[t][0], dO[t][1], bq.x, bq.y);
+                            }
+                        }
+                        release(slot);
+                    }
+                    if (!ok) break;
+                    if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
+                        break;
+                    float *p = reinterpret_cast<float *>(pb);
+    #pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        float sv[4];
+    #pragma unroll
+                        for (int q = 0; q < 4; ++q) sv[q] = facc[t][q] * 16777216.0f;
+                        if (qv == 0) {
+                            sv[0] -= sx0;
+                            sv[1] -= sx1;
+                            sv[2] -= sx0;
+                            sv[3] -= sx1;
+                        }
+                        const int m0 = 2 * c, m1 = 2 * c + 1;
+                        if (m0 < M) {
+                            p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
+                            p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
+                        }
+                        if (m1 < M) {
+                            p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
+                            p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
+                        }
+                    }
                 }
-                if (!ok) break;
-                if (pi >= NB && !dk_warp_wait(&pempty[b], (uint32_t)((pi / NB) - 1) & 1u))
-                    break;
-                float *p = reinterpret_cast<float *>(pb);
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    float sv[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) sv[q] = facc[t][q] * 16777216.0f;
-                    if (qv == 0) {
-                        sv[0] -= sx0;
-                        sv[1] -= sx1;
-                        sv[2] -= sx0;
-                        sv[3] -= sx1;
-                    }
-                    const int m0 = 2 * c, m1 = 2 * c + 1;
-                    if (m0 < M) {
-                        p[((m0 * 16 + cw) * 2 + t) * 16 + g] = sv[0];
-                        p[((m0 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[2];
-                    }
-                    if (m1 < M) {
-                        p[((m1 * 16 + cw) * 2 + t) * 16 + g] = sv[1];
-                        p[((m1 * 16 + cw) * 2 + t) * 16 + g + 8] = sv[3];
-                    }
-                }
-            }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&pfull[b]);
