@@ -250,12 +250,14 @@ def test_batch_matches_single_calls():
 
 
 @pytest.mark.parametrize("fmt", [2, 16])
-def test_long_chain_multiple_items_per_cta(fmt):
+@pytest.mark.parametrize("M", [2, 6])
+def test_long_chain_multiple_items_per_cta(fmt, M):
     """Eight chained 4096 x 4096 layers: 280 items, more than one per CTA, so a
-    CTA holds stages of layer l while its next item waits for layer l."""
+    CTA holds stages of layer l while its next item waits for layer l (at
+    M = 6 the dependent layers convert their X once per launch)."""
     import torch
     import ternary_weight_03_b200 as tl
-    M, D, depth = 2, 4096, 8
+    D, depth = 4096, 8
     Ts = [synth.trits(80 + i, D, D) for i in range(depth)]
     X0 = synth.activations(90, M, D)
     alphas = [0.02] * depth
@@ -318,6 +320,66 @@ def test_decode_step_210_layers_sampled(fmt, M):
         ns = np.concatenate([rng.integers(0, N, 24), [N - 1]])
         ref = o.linear_at(T, X, sp[1], ms, ns)
         tol = oracle.tolerance(ref, X[ms], sp[1])
+        assert (np.abs(Y[ms, ns] - ref) <= tol).all(), f"layer seed {seed}"
+
+
+@pytest.mark.parametrize("fmt,M", [(2, 1), (2, 8), (16, 1), (16, 8)])
+def test_fused_decode_step_sampled(fmt, M):
+    """The decode step as the bench's fused variant runs it, in one batch
+    launch: per decoder block Q, K and V on one X (one conversion), O on its
+    own X, gate and up writing the two halves of one buffer, and the down
+    projection reading silu(gate) * up from it (TL_LAYER_SWIGLU_INPUT, so it
+    waits for that block's gate and up only).  Sampled outputs of every
+    layer against the oracle: the down projections on fp16(silu(g) u)
+    formed here in double from the stored gate and up outputs."""
+    import torch
+    import ternary_weight_03_b200 as tl
+    specs, checks = [], []
+    for blk in range(30):
+        base = 1000 + 7 * blk
+        xa, xo, xf = (synth.activations(base + j, M, 3072) for j in (0, 3, 4))
+        dxa, dxo, dxf = (torch.from_numpy(v).cuda() for v in (xa, xo, xf))
+        gu = torch.full((M, 2 * 8192), float("nan"), dtype=torch.float16, device="cuda")
+        for j, (K, N) in enumerate(DECODE_LAYER):
+            seed = base + j
+            dP = torch.from_numpy(tl.pack(fmt, synth.trits(seed, N, K))).cuda()
+            a = synth.alpha_for(seed)
+            if j < 3:
+                Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+                specs.append((dP, a, dxa, K, Y))
+                checks.append((seed, K, N, a, xa, Y, None))
+            elif j == 3:
+                Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+                specs.append((dP, a, dxo, K, Y))
+                checks.append((seed, K, N, a, xo, Y, None))
+            elif j < 6:
+                Y = gu[:, :8192] if j == 4 else gu[:, 8192:]
+                specs.append((dP, a, dxf, K, Y))
+                checks.append((seed, K, N, a, xf, Y, None))
+            else:
+                Y = torch.full((M, N), float("nan"), dtype=torch.float16, device="cuda")
+                specs.append((dP, a, gu, K, Y, tl.LAYER_READS_EARLIER | tl.LAYER_SWIGLU_INPUT))
+                checks.append((seed, K, N, a, None, Y, gu))
+    layers = tl.make_layers(fmt, specs)
+    plan, ws = _plan(fmt, layers)
+    tl.gemv_batch_run(plan, flags=tl.FLAG_PDL)
+    assert tl.device_status() == 0
+    o = oracle.get()
+    rng = np.random.default_rng(fmt * 100 + M)
+    for seed, K, N, a, X, Yt, GU in checks:
+        Y = Yt.float().cpu().numpy().astype(np.float64)
+        assert np.isfinite(Y).all(), f"layer seed {seed}"
+        T = synth.trits(seed, N, K)
+        ms = np.concatenate([rng.integers(0, M, 16), [M - 1]])
+        ns = np.concatenate([rng.integers(0, N, 16), [N - 1]])
+        if GU is None:
+            ref = o.linear_at(T, X, a, ms, ns)
+            tol = oracle.tolerance(ref, X[ms], a)
+        else:
+            x = _silu_glu(GU.cpu().numpy(), K).astype(np.float16)
+            ref = o.linear_at(T, x, a, ms, ns)
+            ulp = np.spacing(np.abs(x[ms])).astype(np.float64).sum(axis=1)
+            tol = oracle.tolerance(ref, x[ms], a) + abs(a) * ulp
         assert (np.abs(Y[ms, ns] - ref) <= tol).all(), f"layer seed {seed}"
 
 
@@ -461,16 +523,19 @@ def test_dependent_layer_before_independent_ones(fmt):
 
 
 @pytest.mark.parametrize("fmt", [2, 16])
-def test_interleaved_chains(fmt):
+@pytest.mark.parametrize("M", [2, 5])
+def test_interleaved_chains(fmt, M):
     """Dependencies follow the data: a dependent layer waits for the earlier
     layers whose Y overlaps its X, not for every earlier layer.  Two chains
     interleave (a0, b0, a1 reads a0, b1 reads b0's output plus 500 more
     columns of the same buffer), and a flagged SwiGLU layer whose [gate | up]
     input no layer of the batch writes runs without waiting.  Each layer
-    against the oracle on the inputs as stored; two runs agree bit for bit."""
+    against the oracle on the inputs as stored; two runs agree bit for bit.
+    At M = 5 the dependent layers convert their X once per launch (fp16
+    engine), the SwiGLU layer without waiting for any layer."""
     import torch
     import ternary_weight_03_b200 as tl
-    M, K0 = 2, 3000
+    K0 = 3000
     X0, X1 = synth.activations(130, M, K0), synth.activations(131, M, K0)
     GUc = synth.activations(132, M, 2 * 800)
     Ta0, Tb0 = synth.trits(133, 1000, K0), synth.trits(134, 2000, K0)
