@@ -1865,11 +1865,15 @@ namespace tlk {
 // stage as the integer engine.
 inline int dk_stage_cost(int fmt, int M) { return M <= kDkImmaMaxM ? 1 : (fmt == 2 ? 2 : 3); }
 // Cost per item for a batch of total cost `total` (in integer-engine stages):
-// about four items per SM of a B200, so that the longest-first order leaves a
+// a few items per SM of a B200, so that the longest-first order leaves a
 // short tail, but 4..16 integer-engine stages of cost, so item boundaries
-// (and the epilogue work per item) stay rare.
-inline int dk_item_cost(int64_t total) {
-    const int64_t t = total / (4 * kDkRefSms);
+// (and the epilogue work per item) stay rare.  Three items per SM for 2-bit
+// and four for base 3, whose ALU-bound stages gain nothing from the extra
+// bandwidth the last CTAs of a launch find (measured on batches of the six
+// decode shapes at M = 1, 8 and both: 2-bit both 45.4 -> 43.0 us with three
+// instead of four, the rest unchanged; base 3 slower with fewer items).
+inline int dk_item_cost(int fmt, int64_t total) {
+    const int64_t t = total / ((fmt == 2 ? 3 : 4) * kDkRefSms);
     return t < 4 ? 4 : (t > 16 ? 16 : (int)t);
 }
 // K-parts of a layer: items of about `target` stages, cut at stage
@@ -1919,7 +1923,7 @@ inline DkSchedule dk_schedule(int fmt, int count, const DkHostLayer *in, uint8_t
     for (int l = 0; l < count; ++l)
         total += (int64_t)stages_of(in[l]) * ((in[l].N + kDkRows - 1) / kDkRows) *
                  stage_cost(in[l].M);
-    const int cost = dk_item_cost(total);
+    const int cost = dk_item_cost(fmt, total);
     // fp16-engine items stay at 8 stages or more: their epilogue (M outputs
     // per row) must keep up with the consumers.  A layer that waits for the
     // earlier layers starts alone, so its items are sized to spread it over

@@ -151,7 +151,7 @@ def _ws_expected(layers, fmt=2):
     # relative cost of a stage: fp16 engine x2 (2-bit) or x3 (base 3)
     cm = lambda d: 1 if d["M"] <= 2 else (2 if fmt == 2 else 3)
     total = sum(stg(d) * -(-d["N"] // 256) * cm(d) for d in layers)
-    cost = min(16, max(4, total // (4 * 148)))  # cost per item
+    cost = min(16, max(4, total // ((3 if fmt == 2 else 4) * 148)))  # cost per item
     seen = set()
     for d in layers:
         stages = stg(d)
