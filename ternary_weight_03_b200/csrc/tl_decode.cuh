@@ -91,7 +91,7 @@ constexpr int kDkWarps = kDkFirstCons + kDkConsumers;  // 24
 constexpr int kDkThreads = 32 * kDkWarps;              // 768
 constexpr int kDkMaxStages = 6;
 constexpr int kDkQueue = 16;
-constexpr int kDkMaxPartBufs = 4;  // consumer -> epilogue buffers (2 when they are large)
+constexpr int kDkMaxPartBufs = 4;  // consumer -> epilogue buffers (2 when large, in long launches)
 constexpr int kDkImmaMaxM = 2;                          // exact integer engine up to 2 tokens
 constexpr int kDkRefSms = 148;                          // scheduling reference: SMs of a B200
 constexpr int kDkMaxItemStages = 64;                    // s32 sums of an item stay exact
@@ -207,6 +207,7 @@ struct DkArgs {
     int maxM;
     int chained;  // 1: some layer reads an earlier layer's output; 2: and one has a SwiGLU input
     int drop_arrive;  // failure-detection hook (debug library only), else 0
+    int wide;         // four consumer -> epilogue buffers even for large partials
 };
 
 struct DkQEntry {
@@ -225,10 +226,10 @@ struct DkQEntry {
 
 struct DkLayout {
     uint32_t ns, nbufs, slot_b, parts, w_off, st_off, part_off, q_off, bar_off, total;
-    __host__ __device__ DkLayout(int fmt, int maxM) {
+    __host__ __device__ DkLayout(int fmt, int maxM, bool wide) {
         slot_b = dk_slot_b(fmt, maxM) + kDkMetaBytes;  // [meta][B]
         parts = dk_part_bytes(maxM);
-        nbufs = parts <= 8192u ? (uint32_t)kDkMaxPartBufs : 2u;
+        nbufs = parts <= 8192u || wide ? (uint32_t)kDkMaxPartBufs : 2u;
         const uint32_t per_stage = (uint32_t)kDkWBytes + slot_b;
         const uint32_t fixed = nbufs * parts + kDkQueue * (uint32_t)sizeof(DkQEntry) +
                                8u * (3u * kDkMaxStages + 2u * kDkQueue + 2u * kDkMaxPartBufs) +
@@ -796,7 +797,7 @@ template <int FMT, bool kGlu>
 __global__ void __launch_bounds__(kDkThreads, 1) decode2_kernel(const __grid_constant__ DkArgs a) {
     constexpr int TS = dk_trits(FMT);  // activations per stage
     extern __shared__ __align__(1024) uint8_t dk_smem_raw[];
-    const DkLayout lay(FMT, a.maxM);
+    const DkLayout lay(FMT, a.maxM, a.wide != 0);
     const int NS = (int)lay.ns;
     // 1024-byte alignment for the 128-byte swizzle of the weight boxes
     uint8_t *smem = dk_smem_raw + ((1024u - (smem_u32(dk_smem_raw) & 1023u)) & 1023u);
@@ -2135,6 +2136,10 @@ inline DkArgs dk_args(void *ws, int count, int total_items, int total_units, int
     a.maxM = maxM;
     a.chained = chained;
     a.drop_arrive = 0;
+    // short launches with large partials (M > 4, under 8 items per SM):
+    // their epilogues and tail, not the stream, set the pace, so four
+    // epilogue buffers pay for one stage less of ring
+    a.wide = maxM > 4 && total_items < 8 * kDkRefSms ? 1 : 0;
     return a;
 }
 
@@ -2153,8 +2158,10 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     std::call_once(once[dev], [dev] {
         uint32_t most = 0;
         for (int m = 1; m <= 8; ++m) {
-            const uint32_t t = DkLayout(FMT, m).total;
-            most = t > most ? t : most;
+            for (int w = 0; w < 2; ++w) {
+                const uint32_t t = DkLayout(FMT, m, w != 0).total;
+                most = t > most ? t : most;
+            }
         }
         attr_err[dev] = cudaFuncSetAttribute(decode2_kernel<FMT, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
@@ -2169,7 +2176,7 @@ inline int launch_decode2(const DkArgs &a, int num_sms, bool pdl, cudaStream_t s
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.total_items < num_sms ? a.total_items : num_sms));
     cfg.blockDim = dim3(kDkThreads);
-    cfg.dynamicSmemBytes = DkLayout(FMT, a.maxM).total;
+    cfg.dynamicSmemBytes = DkLayout(FMT, a.maxM, a.wide != 0).total;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
