@@ -99,20 +99,22 @@ __device__ __forceinline__ void decode2_exact(uint32_t w, uint32_t *out) {
 
 // Base-3 digits of the four bytes of w (byte = d0 + 3 d1 + 9 d2 + 27 d3 + 81 d4):
 // E[i] holds digit i of byte b in its byte lane b.  The bytes are spread over
-// two registers of 16-bit lanes; for v <= 255, floor(v / 3) = (v * 171) >> 9
-// and v * 171 < 2^16, so both lanes divide at once without a carry between them.
+// two registers of 16-bit lanes, so one IMAD divides two bytes at once.
 __device__ __forceinline__ void digits3_word(uint32_t w, uint32_t (&E)[5]) {
-    uint32_t lo = w & 0x00FF00FFu;         // bytes 0 and 2
-    uint32_t hi = (w >> 8) & 0x00FF00FFu;  // bytes 1 and 3
+    uint32_t lo = prmt(w, 0u, 0x4240u);  // bytes 0 and 2 in 16-bit lanes
+    uint32_t hi = prmt(w, 0u, 0x4341u);  // bytes 1 and 3
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t qlo = ((lo * 171u) >> 9) & 0x007F007Fu;
-        const uint32_t qhi = ((hi * 171u) >> 9) & 0x007F007Fu;
-        E[i] = (lo - 3u * qlo) | ((hi - 3u * qhi) << 8);  // v mod 3, lane by lane
+        // floor(v / 3) = floor(85 (v + 1) / 256) for the valid codes v < 243
+        // (85 (v + 1) < 2^16): the product's high byte, moved back into the
+        // lane's low byte by the PRMT
+        const uint32_t qlo = prmt(lo * 85u + 0x00550055u, 0u, 0x4341u);
+        const uint32_t qhi = prmt(hi * 85u + 0x00550055u, 0u, 0x4341u);
+        E[i] = prmt(lo - 3u * qlo, hi - 3u * qhi, 0x6240u);  // v mod 3, byte by byte
         lo = qlo;
         hi = qhi;
     }
-    E[4] = lo | (hi << 8);
+    E[4] = prmt(lo, hi, 0x6240u);
 }
 
 // Exact decode of K-step J (trits 64 J .. 64 J + 63) of a 320-trit block of
