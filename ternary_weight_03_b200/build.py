@@ -26,7 +26,7 @@ LIB = PKG / "libternary.so"
 DEBUG_LIB = PKG / "libternary_debug.so"
 SOURCES = [CSRC / "tl_device.cu", CSRC / "tl_host.cpp"]
 EXPORTS = CSRC / "exports.map"
-DEPENDS = SOURCES + sorted(CSRC.glob("*.cuh")) + [INCLUDE / "tl.h", EXPORTS]
+DEPENDS = SOURCES + sorted(CSRC.glob("*.cuh")) + [INCLUDE / "tl.h", INCLUDE / "tl_debug.h", EXPORTS]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
               "-shared", "-Xcompiler", "-fPIC", "-Xcompiler", "-pthread",

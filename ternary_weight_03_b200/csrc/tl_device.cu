@@ -8,6 +8,9 @@
 #include <cuda_runtime.h>
 
 #include "tl.h"
+#ifdef TL_DEBUG_HOOKS
+#include "tl_debug.h"
+#endif
 #include "tl_common.cuh"
 #include "tl_gemv.cuh"
 #include "tl_gemm.cuh"
@@ -329,6 +332,26 @@ int tl_gemv_batch_run(const tl_gemv_plan *plan, unsigned int flags, void *stream
                : tlk::launch_decode2<16>(da, dev->num_sms, pdl, (cudaStream_t)stream,
                                          &t_last_cuda_error);
 }
+
+#ifdef TL_DEBUG_HOOKS
+int tl_debug_batch_items(int fmt, int count, const tl_gemv_layer *layers, void *items,
+                         size_t items_bytes, int *n_items) {
+    static_assert(sizeof(tlk::DkItemRec) == TL_DEBUG_ITEM_BYTES, "record size");
+    if (!n_items || (!items && items_bytes > 0)) return TL_ERR_INVALID_ARG;
+    std::vector<tlk::DkHostLayer> h(count > 0 && count <= TL_GEMV_BATCH_MAX ? count : 0);
+    int rc = batch_layers(fmt, count, layers, h.data());
+    if (rc != TL_OK) return rc;
+    // a workspace base that is never dereferenced: the table only holds addresses
+    uint8_t *ws = reinterpret_cast<uint8_t *>((uintptr_t)1 << 40);
+    std::vector<tlk::DkItemRec> recs;
+    std::vector<tlk::DkUnitRec> units;
+    tlk::dk_schedule(fmt, count, h.data(), ws, &recs, &units);
+    const size_t n = std::min(recs.size(), items_bytes / sizeof(tlk::DkItemRec));
+    if (n) std::memcpy(items, recs.data(), n * sizeof(tlk::DkItemRec));
+    *n_items = (int)recs.size();
+    return TL_OK;
+}
+#endif
 
 int tl_device_status(void *stream) {
     cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
